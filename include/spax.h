@@ -1,0 +1,237 @@
+/*
+ * spax.h — C ABI of libspax.so: three-tier, activation-sparse decode GEMV on B200 (sm_100a).
+ *
+ * What the library computes (one token, batch-one decode, one projection y = W·x):
+ *   Every weight column j of W (d_out × d_in) is put in one of three tiers by the magnitude of
+ *   the activation x_j: skipped (|x_j| closest to zero), read as a 2-bit approximation (smaller
+ *   |x_j|), or read in its original format (largest |x_j|).
+ *   Source: "SpAx: Activation Sparsity with Weight Approximation for Faster LLM Decoding on
+ *   Offloaded Weights" (arXiv 2610.02598), Abstract; eigenradar commentary on SpAx, section
+ *   "The route outside GPU memory" (original / two-bit approximate / unread tier per column).
+ *   The tier rules (threshold, TopK, TopK-Guided ±δ clip) follow "TopK-Guided: Adaptive,
+ *   Budget-Aware Activation Sparsity for Efficient LLM Inference" (arXiv 2610.01763),
+ *   Abstract, §1 and §2.1; the block budgets follow its §2.2.
+ *
+ * Conventions shared by every entry point
+ *   - Pointers named d_* (and every tensor argument of a device call) are DEVICE pointers;
+ *     pointers named h_* are HOST pointers. The caller owns all memory; the library never
+ *     allocates and keeps no state except a per-device cache of the SM count.
+ *   - Device calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = the
+ *     legacy default stream) and never synchronise the host. Kernels are launched with the
+ *     programmatic-dependent-launch attribute, so consecutive spax calls on one stream (and in
+ *     a captured CUDA graph) overlap launch latency; every kernel waits for its predecessor
+ *     before touching global memory.
+ *   - The returned spax_status reports argument/shape errors (nothing is launched) and launch
+ *     errors (SPAX_ERR_CUDA). Data-dependent errors found on the device (non-finite input,
+ *     malformed index lists, a pipeline wait that ran out) are written to *d_status (an int32
+ *     on the device, may be NULL) as a spax_status value; the caller reads it after a sync.
+ *     A kernel never clears *d_status; the caller zeroes it.
+ *   - Tier codes: 0 = skip, 1 = approximate (2-bit), 2 = full (original format).
+ *   - Compacted column lists are in ascending column order.
+ *
+ * Packed weight layout (produced by spax_pack_weights, read by spax_tiered_gemv)
+ *   The dense matrix W arrives row-major [d_out][d_in] bf16 (the nn.Linear layout). Packing
+ *   makes every column contiguous, so a selected column is one contiguous run in HBM.
+ *   d_out must be a multiple of 128 (the quantisation group).
+ *   full pool, SPAX_FULL_BF16: W^T as bf16 [d_in][d_out]; column stride 2*d_out bytes.
+ *   full pool, SPAX_FULL_INT4_G128: per column, ceil(d_out/1024) records of 528 bytes:
+ *       512 bytes of 4-bit codes for 1024 rows (byte b holds row 2b in its low nibble and row
+ *       2b+1 in its high nibble; a nibble stores u = q + 8 for the signed code q in [-8, 7]),
+ *       then 8 bf16 scales, one per 128-row group. Value = q * scale (symmetric).
+ *   approx pool (2-bit, asymmetric, group 128): per column, ceil(d_out/512) records of 144
+ *       bytes: 128 bytes of 2-bit codes for 512 rows (byte b holds rows 4b..4b+3, row r at bits
+ *       2*(r%4)), then 4 little-endian uint32 words, word g = bf16 scale bits | (bf16 min bits
+ *       << 16) for the record's group g. Value = min + q * scale, q in [0, 3].
+ *   Rows past d_out in a column's last record are padding: 2-bit code 0 with scale = min = 0;
+ *   int4 nibble 8 (q = 0) with scale 0.
+ */
+#ifndef SPAX_H_
+#define SPAX_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SPAX_ABI_VERSION 1
+
+typedef enum {
+  SPAX_OK = 0,
+  SPAX_ERR_ARG = 1,        /* bad argument (NULL pointer, negative size, bad enum, bad params) */
+  SPAX_ERR_SHAPE = 2,      /* unsupported shape (d_out % 128 != 0, size over a stated limit) */
+  SPAX_ERR_WORKSPACE = 3,  /* workspace pointer NULL or ws_bytes too small */
+  SPAX_ERR_CUDA = 4,       /* a CUDA runtime call or launch failed */
+  SPAX_ERR_NONFINITE = 5,  /* device: an input activation was NaN or Inf */
+  SPAX_ERR_TIMEOUT = 6,    /* device: a bounded pipeline wait ran out (a library bug) */
+  SPAX_ERR_INDEX = 7       /* device: counts or a column index out of range */
+} spax_status;
+
+typedef enum { SPAX_FULL_BF16 = 0, SPAX_FULL_INT4_G128 = 1 } spax_full_fmt;
+
+typedef enum { SPAX_MASK_THRESHOLD = 0, SPAX_MASK_TOPK = 1, SPAX_MASK_GUIDED = 2 } spax_mask_mode;
+
+typedef enum { SPAX_OP_TIERED_GEMV = 0, SPAX_OP_DENSE_GEMV = 1, SPAX_OP_CALIBRATE = 2 } spax_op;
+
+/* Largest d_in a mask call accepts (the activation vector lives in one CTA's shared memory). */
+#define SPAX_MASK_MAX_DIN 49152
+
+/*
+ * Tier-rule parameters for spax_build_mask.
+ *   THRESHOLD (TEAL-style; TopK-Guided Abstract and §1): skip if |x| < t_skip, approximate if
+ *     t_skip <= |x| < t_full, full otherwise. Requires 0 <= t_skip <= t_full.
+ *   TOPK (WINA-style fixed count; TopK-Guided Abstract and §1): columns ranked by |x|, largest
+ *     first, ties broken by the lower column index first; the first k_full ranks are full, the
+ *     next k_approx approximate, the rest skipped. Requires k_full, k_approx >= 0 and
+ *     k_full + k_approx <= d_in.
+ *   GUIDED (TopK-Guided §2.1): the natural counts n1 = #{|x| < t_skip} and n2 = #{|x| < t_full}
+ *     are clipped into the bands [ceil((s-δ)d), floor((s+δ)d)] around the skip target
+ *     s = s_skip_bp/1e4 and the skip-or-approximate target s = s_below_full_bp/1e4
+ *     (δ = delta_bp/1e4), giving m1 <= m2; then TOPK with k_full = d - m2,
+ *     k_approx = m2 - m1. All band arithmetic is integer. Requires 0 <= s_skip_bp <=
+ *     s_below_full_bp <= 10000, 0 <= delta_bp <= 10000, and the THRESHOLD requirements.
+ */
+typedef struct {
+  int32_t mode;
+  float t_skip;
+  float t_full;
+  int32_t k_full;
+  int32_t k_approx;
+  int32_t s_skip_bp;
+  int32_t s_below_full_bp;
+  int32_t delta_bp;
+} spax_mask_params;
+
+/* A packed matrix: both pools in device memory, owned by the caller. */
+typedef struct {
+  int32_t d_out;
+  int32_t d_in;
+  int32_t full_fmt;  /* spax_full_fmt */
+  int32_t reserved;
+  const void* d_full;    /* full pool, layout above */
+  const void* d_approx;  /* approx pool, layout above */
+} spax_packed;
+
+/* ABI version (SPAX_ABI_VERSION) and a static string for a status code. */
+int spax_abi_version(void);
+const char* spax_status_string(int status);
+
+/*
+ * Bytes of the two packed pools of a d_out × d_in matrix (host-only, no CUDA call).
+ * Writes *h_full_bytes and *h_approx_bytes (either may be NULL); returns their sum, or 0 for an
+ * invalid shape/format.
+ */
+size_t spax_pack_bytes(int d_out, int d_in, int full_fmt, size_t* h_full_bytes,
+                       size_t* h_approx_bytes);
+
+/*
+ * spax_pack_weights — offline: quantise and re-lay W for the tiered GEMV.
+ * Source: SpAx Abstract ("compressed weight representation"); eigenradar "two-bit approximate"
+ * tier. Quantiser per column and 128-row group, in fp32 with IEEE rounding:
+ *   2-bit: mn, mx = min, max of the group; min = bf16(mn); scale = bf16_rne((mx - mn) / 3);
+ *          q = clamp(rint_even((w - min) / scale), 0, 3), q = 0 when scale == 0.
+ *   int4:  scale = bf16_rne(max|w| / 7); q = clamp(rint_even(w / scale), -8, 7), q = 0 when
+ *          scale == 0.
+ * d_W: row-major [d_out][d_in] bf16 (device). d_full / d_approx: device buffers of at least
+ * spax_pack_bytes() bytes each, fully written (padding included). Returns SPAX_ERR_SHAPE if
+ * d_out % 128 != 0 or d_out, d_in < 1; SPAX_ERR_ARG for NULL pointers or a bad format.
+ */
+spax_status spax_pack_weights(const void* d_W, int d_out, int d_in, int full_fmt, void* d_full,
+                              void* d_approx, void* stream);
+
+/*
+ * spax_calibrate_thresholds — offline: the calibrated |x| thresholds of the threshold and
+ * guided rules (TopK-Guided §2.1 "calibrated threshold", §2.2 calibration pass).
+ * Pools the M = n_tok * d_in values |x| of d_calib_x (row-major [n_tok][d_in] fp32) and, for
+ * s = s_skip_bp/1e4 and s = s_below_full_bp/1e4, returns the order statistic of 0-based rank
+ * min(floor(s*M + 1/2), M - 1) of the ascending |x| values (integer arithmetic). Writes
+ * d_t_out[0] = t_skip and d_t_out[1] = t_full (device fp32). A NaN or Inf input sets
+ * *d_status = SPAX_ERR_NONFINITE (thresholds are then unspecified).
+ * Workspace: spax_workspace_bytes(SPAX_OP_CALIBRATE, 0, d_in) bytes of device memory, any
+ * contents. Requires n_tok, d_in >= 1, n_tok * d_in < 2^31, 0 <= s_*_bp <= 10000.
+ */
+spax_status spax_calibrate_thresholds(const float* d_calib_x, int n_tok, int d_in, int s_skip_bp,
+                                      int s_below_full_bp, float* d_t_out, int32_t* d_status,
+                                      void* d_ws, size_t ws_bytes, void* stream);
+
+/*
+ * spax_build_mask — per token: the tier of every column and the compacted column lists.
+ * Source: SpAx Abstract (three options chosen by activation magnitude); TopK-Guided §2.1
+ * (mask construction in O(d), realised sparsity within ±δ of the target).
+ * d_x: fp32 [d_in] activations. Outputs (device): d_tier uint8 [d_in] (0/1/2),
+ * d_full_idx int32 [d_in] and d_approx_idx int32 [d_in] (the first counts[0] / counts[1]
+ * entries are written, ascending), d_counts int32 [4] = {n_full, n_approx, n1, n2} with n1, n2
+ * the natural threshold counts (0 for TOPK). A NaN/Inf in x sets *d_status =
+ * SPAX_ERR_NONFINITE, every tier to 0 and the counts to 0. h_params is a host pointer, read
+ * during the call. d_in <= SPAX_MASK_MAX_DIN. One CTA; no workspace.
+ */
+spax_status spax_build_mask(const float* d_x, int d_in, const spax_mask_params* h_params,
+                            uint8_t* d_tier, int32_t* d_full_idx, int32_t* d_approx_idx,
+                            int32_t* d_counts, int32_t* d_status, void* stream);
+
+/*
+ * spax_tiered_gemv — per token: y = Σ_{j in full} x_j W[:,j] + Σ_{j in approx} x_j deq2(W)[:,j].
+ * Source: SpAx Abstract (read original weights for the largest |x|, approximate weights for
+ * smaller, skip the rest); eigenradar commentary (bytes moved per token; reconstruction of
+ * two-bit approximations costs GPU time).
+ * h_W: host pointer to the packed-matrix descriptor (device pools). d_x fp32 [d_in];
+ * d_full_idx / d_approx_idx / d_counts as written by spax_build_mask (the kernel reads
+ * counts on the device; no host sync). d_y fp32 [d_out] (device), fully written.
+ * Accumulation is fp32, split over CTAs, then reduced in a fixed order (bit-reproducible for a
+ * given GPU model and shape). Workspace: spax_workspace_bytes(SPAX_OP_TIERED_GEMV, d_out, d_in)
+ * bytes, ZEROED BEFORE FIRST USE (it holds arrival counters that every completed call leaves
+ * at zero; zero it again after a device error). Counts outside [0, d_in] or an index outside
+ * [0, d_in) set *d_status = SPAX_ERR_INDEX; such a column contributes zero.
+ * Calls that share a workspace must not run concurrently.
+ */
+spax_status spax_tiered_gemv(const spax_packed* h_W, const float* d_x, const int32_t* d_full_idx,
+                             const int32_t* d_approx_idx, const int32_t* d_counts, float* d_y,
+                             int32_t* d_status, void* d_ws, size_t ws_bytes, void* stream);
+
+/*
+ * spax_dense_gemv — the same-GPU dense baseline: y = W x over every column, read from the
+ * bf16 full pool (W^T [d_in][d_out]) with the same kernel family as spax_tiered_gemv.
+ * Source: eigenradar commentary (comparisons use dense decoding in the same weight format).
+ * Workspace: spax_workspace_bytes(SPAX_OP_DENSE_GEMV, d_out, d_in) bytes, zeroed before first
+ * use (same rule as spax_tiered_gemv). d_out % 128 == 0.
+ */
+spax_status spax_dense_gemv(const void* d_Wt, const float* d_x, float* d_y, int d_out, int d_in,
+                            int32_t* d_status, void* d_ws, size_t ws_bytes, void* stream);
+
+/*
+ * Device workspace bytes an op needs for a shape on the CURRENT device (the split count
+ * depends on its SM count). Returns 0 for an invalid op or shape.
+ */
+size_t spax_workspace_bytes(int op, int d_out, int d_in);
+
+/*
+ * Host-only: the split-K factor S and row tile R the tiered/dense GEMV uses for a shape on the
+ * current device (for reporting and tests). Returns SPAX_ERR_SHAPE/ARG on a bad shape.
+ */
+spax_status spax_gemv_plan(int op, int d_out, int d_in, int full_fmt, int32_t* h_splits,
+                           int32_t* h_row_tile);
+
+/*
+ * spax_block_budgets — host-only: sensitivity-aware per-block sparsity (TopK-Guided §2.2:
+ * above-average-sensitivity blocks get less sparsity, λ sets the redistribution, results are
+ * clamped to [lo, hi], the global budget is kept). With σ̄ the mean of h_sens:
+ *   s_b = clamp(s * (1 - λ (σ_b/σ̄ - 1)) + c, lo, hi), c chosen so that mean_b s_b = s.
+ * h_sens: n_blocks positive sensitivities; writes h_s_out[n_blocks]. Requires lo <= s <= hi,
+ * 0 <= lo <= hi <= 1, λ >= 0, n_blocks >= 1.
+ */
+spax_status spax_block_budgets(const double* h_sens, int n_blocks, double s, double lambda,
+                               double lo, double hi, double* h_s_out);
+
+/*
+ * Host-only byte account of one tiered GEMV (eigenradar "bytes moved per generated token"):
+ * weight bytes the kernel must read for n_full full and n_approx approximate columns of a
+ * d_out-row matrix: n_full * (2*d_out for bf16 | 0.5*d_out + 2*d_out/128 for int4) +
+ * n_approx * (d_out/4 + 4*d_out/128). Returns 0 on a bad shape.
+ */
+uint64_t spax_weight_bytes(int d_out, int full_fmt, int64_t n_full, int64_t n_approx);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SPAX_H_ */

@@ -1,0 +1,262 @@
+"""CPU oracle of the three-tier decode GEMV (plain C, fp64 accumulation) behind ctypes.
+
+TEST INFRASTRUCTURE ONLY. Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py`` may import this package. The product path (``tiered_weight_gemv_b200``)
+never imports it, and it never imports the product: the two share no code, header, table or
+helper. Inputs come from the seeded generators in ``tiered_weight_gemv_b200.synth``, which hold
+none of the method's arithmetic.
+
+Every function cites the passage it follows (see ``spax_oracle.c`` for the rules written out):
+  * SpAx: Activation Sparsity with Weight Approximation for Faster LLM Decoding on Offloaded
+    Weights — Abstract (three tiers by activation magnitude).
+  * eigenradar commentary on SpAx — "The route outside GPU memory" (original / two-bit / unread
+    tier per column; bytes moved per token).
+  * TopK-Guided: Adaptive, Budget-Aware Activation Sparsity for Efficient LLM Inference —
+    Abstract, §1 (threshold and TopK rules), §2.1 (guided ±δ clip), §2.2 (block budgets).
+
+Every oracle function is pinned by the ``-m "not gpu"`` tests against brute force, closed forms,
+invariants or library routines; none is "parity unpinned" except the readings listed in the
+design notes (the guided three-tier split and the budget formula, pinned only by invariants).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "spax_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libspax_oracle.so")
+
+FULL_BF16 = 0
+FULL_INT4 = 1
+MODE_THRESHOLD = 0
+MODE_TOPK = 1
+MODE_GUIDED = 2
+OK = 0
+ERR_NONFINITE = 5
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (IEEE fp32 steps: no fast-math, no FMA contraction)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.run(
+            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
+             "-Wall", "-o", tmp, _SRC, "-lm"],
+            check=True,
+        )
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+_lib = None
+
+
+def _L():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        i32, i64, f32, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_double
+        lib.oracle_tiers.argtypes = [P, i32, i32, f32, f32, i32, i32, i32, i32, i32, P, P, P, P]
+        lib.oracle_tiers.restype = i32
+        lib.oracle_quant2_group.argtypes = [P, i32, P, P, P]
+        lib.oracle_quant4_group.argtypes = [P, i32, P, P]
+        lib.oracle_pack.argtypes = [P, i32, i32, i32, P, P]
+        lib.oracle_pack.restype = i32
+        lib.oracle_pack_column.argtypes = [P, i32, i32, i32, i32, P, P]
+        lib.oracle_pack_column.restype = i32
+        lib.oracle_full_col_bytes.argtypes = [i32, i32]
+        lib.oracle_full_col_bytes.restype = i64
+        lib.oracle_approx_col_bytes.argtypes = [i32]
+        lib.oracle_approx_col_bytes.restype = i64
+        lib.oracle_full_value.argtypes = [P, i32, i32]
+        lib.oracle_full_value.restype = f64
+        lib.oracle_approx_value.argtypes = [P, i32]
+        lib.oracle_approx_value.restype = f64
+        lib.oracle_tiered_gemv.argtypes = [P, P, i32, i32, i32, P, P, P, i32, P]
+        lib.oracle_tiered_gemv.restype = i32
+        lib.oracle_dense_gemv.argtypes = [P, i32, i32, P, P, i32, P]
+        lib.oracle_dense_gemv.restype = i32
+        lib.oracle_calibrate.argtypes = [P, i64, i32, i32, P]
+        lib.oracle_calibrate.restype = i32
+        lib.oracle_block_budgets.argtypes = [P, i32, f64, f64, f64, f64, P]
+        lib.oracle_block_budgets.restype = i32
+        lib.oracle_weight_bytes.argtypes = [i32, i32, i64, i64]
+        lib.oracle_weight_bytes.restype = ctypes.c_uint64
+        lib.oracle_f32_to_bf16.argtypes = [f32]
+        lib.oracle_f32_to_bf16.restype = ctypes.c_uint16
+        lib.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
+        lib.oracle_bf16_to_f32.restype = f32
+        _lib = lib
+    return _lib
+
+
+def _p(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a), dtype=dtype)
+
+
+# ----------------------------------------------------------------------------- bf16 helpers
+
+def f32_to_bf16_bits(v: float) -> int:
+    """fp32 -> bf16 bits, round to nearest even (written from the definition in C)."""
+    return int(_L().oracle_f32_to_bf16(float(v)))
+
+
+def bf16_bits_to_f32(h: int) -> float:
+    return float(_L().oracle_bf16_to_f32(int(h)))
+
+
+# ----------------------------------------------------------------------------- tier rule
+
+def tiers(x, mode, *, t_skip=0.0, t_full=0.0, k_full=0, k_approx=0, s_skip_bp=0,
+          s_below_full_bp=0, delta_bp=0):
+    """Tier of every column plus ascending compacted lists (SpAx Abstract; TopK-Guided §1, §2.1).
+
+    Returns (status, tier uint8[d], full_idx int32[n_full], approx_idx int32[n_approx],
+    counts int32[4] = {n_full, n_approx, n1, n2}).
+    """
+    x = _c(x, np.float32)
+    d = x.size
+    tier = np.zeros(d, np.uint8)
+    fi = np.zeros(max(d, 1), np.int32)
+    ai = np.zeros(max(d, 1), np.int32)
+    counts = np.zeros(4, np.int32)
+    st = _L().oracle_tiers(_p(x), d, mode, t_skip, t_full, k_full, k_approx, s_skip_bp,
+                           s_below_full_bp, delta_bp, _p(tier), _p(fi), _p(ai), _p(counts))
+    return st, tier, fi[: counts[0]].copy(), ai[: counts[1]].copy(), counts
+
+
+# ----------------------------------------------------------------------------- quantisers
+
+def quant2_group(w_bits):
+    """2-bit asymmetric quantiser of one group of bf16 values (given as uint16 bits)."""
+    w = _c(w_bits, np.uint16)
+    q = np.zeros(w.size, np.uint8)
+    sb = np.zeros(1, np.uint16)
+    mb = np.zeros(1, np.uint16)
+    _L().oracle_quant2_group(_p(w), w.size, _p(q), _p(sb), _p(mb))
+    return q, int(sb[0]), int(mb[0])
+
+
+def quant4_group(w_bits):
+    """int4 symmetric quantiser of one group of bf16 values (given as uint16 bits)."""
+    w = _c(w_bits, np.uint16)
+    q = np.zeros(w.size, np.int8)
+    sb = np.zeros(1, np.uint16)
+    _L().oracle_quant4_group(_p(w), w.size, _p(q), _p(sb))
+    return q, int(sb[0])
+
+
+# ----------------------------------------------------------------------------- packing
+
+def full_col_bytes(d_out: int, fmt: int) -> int:
+    return int(_L().oracle_full_col_bytes(d_out, fmt))
+
+
+def approx_col_bytes(d_out: int) -> int:
+    return int(_L().oracle_approx_col_bytes(d_out))
+
+
+def pack(W_bits, fmt: int):
+    """Pack a row-major bf16 matrix (uint16 bits [d_out, d_in]) into (full, approx) byte pools."""
+    W = _c(W_bits, np.uint16)
+    d_out, d_in = W.shape
+    full = np.zeros(full_col_bytes(d_out, fmt) * d_in, np.uint8)
+    approx = np.zeros(approx_col_bytes(d_out) * d_in, np.uint8)
+    st = _L().oracle_pack(_p(W), d_out, d_in, fmt, _p(full), _p(approx))
+    if st != OK:
+        raise ValueError(f"oracle_pack status {st}")
+    return full, approx
+
+
+def pack_column(W_bits, fmt: int, j: int):
+    """Pack one column j; returns its (full column bytes, approx column bytes)."""
+    W = _c(W_bits, np.uint16)
+    d_out, d_in = W.shape
+    fc = np.zeros(full_col_bytes(d_out, fmt), np.uint8)
+    ac = np.zeros(approx_col_bytes(d_out), np.uint8)
+    st = _L().oracle_pack_column(_p(W), d_out, d_in, fmt, j, _p(fc), _p(ac))
+    if st != OK:
+        raise ValueError(f"oracle_pack_column status {st}")
+    return fc, ac
+
+
+def full_value(full_col, fmt: int, r: int) -> float:
+    fc = _c(full_col, np.uint8)
+    return float(_L().oracle_full_value(_p(fc), fmt, r))
+
+
+def approx_value(approx_col, r: int) -> float:
+    ac = _c(approx_col, np.uint8)
+    return float(_L().oracle_approx_value(_p(ac), r))
+
+
+# ----------------------------------------------------------------------------- products
+
+def tiered_gemv(full, approx, fmt, d_out, d_in, x, tier, rows=None):
+    """fp64 tiered product from the oracle's packed pools (SpAx Abstract; eigenradar)."""
+    full = _c(full, np.uint8)
+    approx = _c(approx, np.uint8)
+    x = _c(x, np.float32)
+    tier = _c(tier, np.uint8)
+    if rows is None:
+        y = np.zeros(d_out, np.float64)
+        st = _L().oracle_tiered_gemv(_p(full), _p(approx), fmt, d_out, d_in, _p(x), _p(tier),
+                                     None, 0, _p(y))
+    else:
+        rows = _c(rows, np.int32)
+        y = np.zeros(rows.size, np.float64)
+        st = _L().oracle_tiered_gemv(_p(full), _p(approx), fmt, d_out, d_in, _p(x), _p(tier),
+                                     _p(rows), rows.size, _p(y))
+    if st != OK:
+        raise ValueError(f"oracle_tiered_gemv status {st}")
+    return y
+
+
+def dense_gemv(W_bits, x, rows=None):
+    """fp64 dense product y = W x from the row-major bf16 matrix (uint16 bits)."""
+    W = _c(W_bits, np.uint16)
+    x = _c(x, np.float32)
+    d_out, d_in = W.shape
+    if rows is None:
+        y = np.zeros(d_out, np.float64)
+        _L().oracle_dense_gemv(_p(W), d_out, d_in, _p(x), None, 0, _p(y))
+    else:
+        rows = _c(rows, np.int32)
+        y = np.zeros(rows.size, np.float64)
+        _L().oracle_dense_gemv(_p(W), d_out, d_in, _p(x), _p(rows), rows.size, _p(y))
+    return y
+
+
+# ----------------------------------------------------------------------------- calibration etc.
+
+def calibrate(X, s_skip_bp: int, s_below_full_bp: int):
+    """Quantile thresholds of pooled |x| (TopK-Guided §2.1 calibrated threshold)."""
+    X = _c(X, np.float32).ravel()
+    t = np.zeros(2, np.float32)
+    st = _L().oracle_calibrate(_p(X), X.size, s_skip_bp, s_below_full_bp, _p(t))
+    return st, float(t[0]), float(t[1])
+
+
+def block_budgets(sens, s, lam, lo=0.05, hi=0.95):
+    """Sensitivity-aware block budgets (TopK-Guided §2.2), exact piecewise-linear solve."""
+    sens = _c(sens, np.float64)
+    out = np.zeros(sens.size, np.float64)
+    st = _L().oracle_block_budgets(_p(sens), sens.size, s, lam, lo, hi, _p(out))
+    if st != OK:
+        raise ValueError(f"oracle_block_budgets status {st}")
+    return out
+
+
+def weight_bytes(d_out: int, fmt: int, n_full: int, n_approx: int) -> int:
+    """Bytes the tiered product reads for one token (eigenradar: bytes moved per token)."""
+    return int(_L().oracle_weight_bytes(d_out, fmt, n_full, n_approx))
