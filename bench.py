@@ -1,0 +1,518 @@
+#!/usr/bin/env python
+"""Benchmark of the three-tier decode GEMV on a Llama-2-7B-shaped decoder block (batch one).
+
+Workload (one step = one pass of the hot path over a batch of synthetic tokens):
+  * one Llama-2-7B-shaped block: q, k, v, o 4096x4096; gate, up 11008x4096; down 4096x11008;
+    bf16 N(0, 0.02) weights (seeded); q/k/v and gate/up packed as one matrix each, so a token
+    runs four sites (attn-in -> qkv, o-in -> o, mlp-in -> gate/up, down-in -> down);
+  * 64 tokens; block inputs fp32 Laplace(0, 1); the down input is SiLU(gate x) * (up x) from the
+    block's own gate/up weights and the mlp input (fp64, prepared once, untimed);
+  * tiers by |x| rank: 40% skipped, 30% 2-bit, 30% bf16 (TopK);
+  * every token reads one of 32 weight replicas (round robin), as a 32-layer stack would, so all
+    launches stream from HBM (inputs larger than L2; no flush needed).
+A step = for each token, for each site: spax_build_mask + spax_tiered_gemv, captured once as a CUDA
+graph (kernels chained with programmatic dependent launch) and replayed.
+
+Metric: us per token per decoder layer (lower is better), plus effective HBM GB/s of the tiered
+GEMV over the bytes it must read, against the dense bf16 GEMV of the same kernel family.
+
+Multi-GPU: replicas only (each rank decodes its own token stream on its own block; no
+collective on the data path). `value` = max-over-ranks step time / (tokens x ranks).
+
+--impl reference runs the CPU oracle (plain C, fp64) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np
+import torch
+import torch.distributed as dist
+
+HIDDEN, INTER = 4096, 11008
+N_TOKENS = 64
+SKIP, APPROX, FULL = 0.4, 0.3, 0.3
+N_REPLICAS = 32
+METRIC = "us/token per decoder layer (three-tier decode GEMV), with effective HBM GB/s vs dense GEMV"
+WORKLOAD = "llama2-7b-block-decode-b1"
+# (name, d_out, d_in, input stream tensor id); q/k/v and gate/up are concatenated along d_out
+SITES = [("qkv", 3 * HIDDEN, HIDDEN, 101), ("o", HIDDEN, HIDDEN, 102),
+         ("gate_up", 2 * INTER, HIDDEN, 103), ("down", HIDDEN, INTER, None)]
+WEIGHT_IDS = {"q": 1, "k": 2, "v": 3, "o": 4, "gate": 5, "up": 6, "down": 7}
+FALLBACK_HBM_GBS = 6650.0
+
+
+def k_counts(d_in: int):
+    kf = int(math.floor(FULL * d_in + 0.5))
+    ka = int(math.floor(APPROX * d_in + 0.5))
+    return kf, ka
+
+
+# ----------------------------------------------------------------------------- distributed
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1 and not dist.is_initialized():
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, ws, local
+
+
+def barrier():
+    if dist.is_initialized():
+        dist.barrier()
+
+
+def max_over_ranks(v: float) -> float:
+    """Max of a per-rank scalar over all ranks (the job's time is its slowest rank's)."""
+    if not dist.is_initialized():
+        return v
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def us_per_token_layer(ms_per_step: float, tokens_per_rank: int, world: int) -> float:
+    """Whole-job us per token per layer: every rank decodes its own tokens through one layer."""
+    return ms_per_step * 1000.0 / (tokens_per_rank * world)
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed regions run."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._thr = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+        self.period = period_s
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thr:
+            self._thr.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- workload
+
+def make_weights(device):
+    from tiered_weight_gemv_b200 import synth
+    W = {n: None for n in WEIGHT_IDS}
+    shapes = {"q": (HIDDEN, HIDDEN), "k": (HIDDEN, HIDDEN), "v": (HIDDEN, HIDDEN),
+              "o": (HIDDEN, HIDDEN), "gate": (INTER, HIDDEN), "up": (INTER, HIDDEN),
+              "down": (HIDDEN, INTER)}
+    for n, tid in WEIGHT_IDS.items():
+        W[n] = synth.weight(*shapes[n], 0, tid, device=device)
+    return {"qkv": torch.cat([W["q"], W["k"], W["v"]], 0).contiguous(), "o": W["o"],
+            "gate_up": torch.cat([W["gate"], W["up"]], 0).contiguous(), "down": W["down"]}
+
+
+def make_inputs(mats, n_tokens, device):
+    from tiered_weight_gemv_b200 import synth
+    xs = {}
+    for name, d_out, d_in, tid in SITES:
+        if tid is not None:
+            xs[name] = synth.laplace((n_tokens, d_in), 0, tid, device=device)
+    gu = mats["gate_up"].to(torch.float64) @ xs["gate_up"].to(torch.float64).T  # [2*INTER, T]
+    xs["down"] = synth.silu_gated(gu[:INTER].T, gu[INTER:].T).contiguous()
+    return xs
+
+
+def algorithmic_bytes(d_out, d_in, kf, ka):
+    """Bytes one tiered GEMV must move: selected weights (+ scales), the gathered x entries, the
+    two index lists and the output vector."""
+    from tiered_weight_gemv_b200 import spax
+    return spax.spax_weight_bytes(d_out, spax.FULL_BF16, kf, ka) + (kf + ka) * 8 + d_out * 4 + 16
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def time_graph(g, steps, warmup, stream):
+    """Mean ms per replay of graph g over `steps` replays on `stream` (events on that stream)."""
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        barrier()
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for _ in range(steps):
+            g.replay()
+        end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    return start.elapsed_time(end) / steps
+
+
+def run_gpu(args, rank, world, local):
+    from tiered_weight_gemv_b200 import spax
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    n_tok, n_rep = args.tokens, args.replicas
+    mats = make_weights(dev)
+    xs = make_inputs(mats, n_tok, dev)
+    host = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        host = ({n: m.cpu() for n, m in mats.items()}, {n: v.cpu() for n, v in xs.items()})
+
+    # packed replicas (pack once, copy) and per-site buffers
+    packed = {}
+    for name, d_out, d_in, _ in SITES:
+        pm = spax.alloc_packed(d_out, d_in, spax.FULL_BF16, device=dev)
+        spax.spax_pack_weights(mats[name], spax.FULL_BF16, pm)
+        reps = [pm] + [spax.PackedMatrix(d_out, d_in, spax.FULL_BF16, pm.full.clone(),
+                                         pm.approx.clone()) for _ in range(n_rep - 1)]
+        packed[name] = reps
+    torch.cuda.synchronize()
+    del mats
+    buf = {}
+    for name, d_out, d_in, _ in SITES:
+        kf, ka = k_counts(d_in)
+        buf[name] = dict(
+            tier=torch.empty(n_tok, d_in, dtype=torch.uint8, device=dev),
+            fidx=torch.empty(n_tok, d_in, dtype=torch.int32, device=dev),
+            aidx=torch.empty(n_tok, d_in, dtype=torch.int32, device=dev),
+            counts=torch.empty(n_tok, 4, dtype=torch.int32, device=dev),
+            y=torch.empty(n_tok, d_out, dtype=torch.float32, device=dev),
+            yd=torch.empty(n_tok, d_out, dtype=torch.float32, device=dev),
+            status=torch.zeros(1, dtype=torch.int32, device=dev),
+            ws=spax.alloc_workspace(spax.OP_TIERED_GEMV, d_out, d_in, device=dev),
+            dws=spax.alloc_workspace(spax.OP_DENSE_GEMV, d_out, d_in, device=dev),
+            prm=spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka),
+            desc=[pm.desc() for pm in packed[name]],
+            kf=kf, ka=ka)
+
+    def step_tiered(mask=True, gemv=True, sites=None):
+        for t in range(n_tok):
+            for name, d_out, d_in, _ in SITES:
+                if sites is not None and name not in sites:
+                    continue
+                b = buf[name]
+                if mask:
+                    spax.spax_build_mask(xs[name][t], b["prm"], b["tier"][t], b["fidx"][t],
+                                         b["aidx"][t], b["counts"][t], b["status"])
+                if gemv:
+                    pm = packed[name][t % n_rep]
+                    spax.spax_tiered_gemv(pm, xs[name][t], b["fidx"][t], b["aidx"][t],
+                                          b["counts"][t], b["y"][t], b["status"], b["ws"],
+                                          desc=b["desc"][t % n_rep])
+
+    def step_dense(sites=None):
+        for t in range(n_tok):
+            for name, d_out, d_in, _ in SITES:
+                if sites is not None and name not in sites:
+                    continue
+                b = buf[name]
+                spax.spax_dense_gemv(packed[name][t % n_rep].full, xs[name][t], b["yd"][t],
+                                     d_out, d_in, b["status"], b["dws"])
+
+    stream = torch.cuda.Stream(device=dev)
+    graphs = {}
+    with torch.cuda.stream(stream):
+        step_tiered()  # eager run: fills the lists used by the GEMV-only graphs
+        step_dense()
+    torch.cuda.synchronize()
+    for name, *_ in SITES:
+        st = int(buf[name]["status"].item())
+        if st != 0:
+            raise RuntimeError(f"device status {st} ({spax.status_string(st)}) at site {name}")
+
+    def capture(fn, *a, **k):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn(*a, **k)
+        return g
+
+    graphs["tiered"] = capture(step_tiered)
+    graphs["dense"] = capture(step_dense)
+    for name, *_ in SITES:
+        graphs["gemv_" + name] = capture(step_tiered, mask=False, gemv=True, sites=[name])
+        graphs["mask_" + name] = capture(step_tiered, mask=True, gemv=False, sites=[name])
+        graphs["dense_" + name] = capture(step_dense, sites=[name])
+
+    res = {}
+    sampler = ClockSampler(local)
+    with sampler:
+        res["tiered"] = max_over_ranks(time_graph(graphs["tiered"], args.steps, args.warmup, stream))
+        res["dense"] = max_over_ranks(time_graph(graphs["dense"], args.steps, args.warmup, stream))
+        for name, *_ in SITES:
+            res["gemv_" + name] = max_over_ranks(
+                time_graph(graphs["gemv_" + name], args.steps, args.warmup, stream))
+            res["mask_" + name] = max_over_ranks(
+                time_graph(graphs["mask_" + name], args.steps, args.warmup, stream))
+            res["dense_" + name] = max_over_ranks(
+                time_graph(graphs["dense_" + name], args.steps, args.warmup, stream))
+        # end to end: host inputs in, host outputs out, through the same C-ABI calls
+        xin = {n: xs[n].cpu().pin_memory() for n in xs}
+        yout = {n: torch.empty(buf[n]["y"].shape, dtype=torch.float32).pin_memory() for n in xs}
+        h2d = sum(v.numel() * 4 for v in xin.values())
+        d2h = sum(v.numel() * 4 for v in yout.values())
+
+        def e2e_once():
+            for n in xs:
+                xs[n].copy_(xin[n], non_blocking=True)
+            graphs["tiered"].replay()
+            for n in xs:
+                yout[n].copy_(buf[n]["y"], non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                e2e_once()
+            torch.cuda.synchronize()
+            barrier()
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            for _ in range(args.steps):
+                e2e_once()
+            s1.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+        res["e2e"] = max_over_ranks(s0.elapsed_time(s1) / args.steps)
+    for name, *_ in SITES:
+        st = int(buf[name]["status"].item())
+        if st != 0:
+            raise RuntimeError(f"device status {st} after timing at site {name}")
+        if not torch.isfinite(buf[name]["y"]).all():
+            raise RuntimeError(f"non-finite output at site {name}")
+
+    launches_per_step = n_tok * len(SITES) * 2
+    sites = {}
+    tot_bytes = tot_ms = 0.0
+    for name, d_out, d_in, _ in SITES:
+        b = buf[name]
+        by = algorithmic_bytes(d_out, d_in, b["kf"], b["ka"])
+        ms = res["gemv_" + name]
+        tot_bytes += by * n_tok
+        tot_ms += ms
+        S, R = spax.spax_gemv_plan(spax.OP_TIERED_GEMV, d_out, d_in)
+        sites[name] = {"d_out": d_out, "d_in": d_in, "n_full": b["kf"], "n_approx": b["ka"],
+                       "gemv_us": round(ms * 1000 / n_tok, 3),
+                       "mask_us": round(res["mask_" + name] * 1000 / n_tok, 3),
+                       "bytes_per_launch": by,
+                       "gemv_GBps": round(by * n_tok / (ms * 1e-3) / 1e9, 1),
+                       "dense_us": round(res["dense_" + name] * 1000 / n_tok, 3),
+                       "dense_GBps": round(2 * d_out * d_in * n_tok / (res["dense_" + name] * 1e-3) / 1e9, 1),
+                       "splits": S, "row_tile": R}
+    return res, sites, tot_bytes, tot_ms, launches_per_step, h2d, d2h, sampler.summary(), host
+
+
+def fit_c0_bw(points):
+    """Least-squares time = c0 + bytes / BW over (bytes, us) points: the fixed per-launch cost and
+    the streaming rate (the byte-account method of the ByteCross abstract)."""
+    b = np.array([p[0] for p in points], np.float64)
+    t = np.array([p[1] for p in points], np.float64)
+    A = np.stack([np.ones_like(b), b], 1)
+    (c0, inv_bw), *_ = np.linalg.lstsq(A, t, rcond=None)
+    pred = A @ np.array([c0, inv_bw])
+    ss = float(((t - t.mean()) ** 2).sum())
+    r2 = 1.0 - float(((t - pred) ** 2).sum()) / ss if ss > 0 else 1.0
+    return {"c0_us": round(float(c0), 3), "GBps": round(1e-3 / inv_bw, 1) if inv_bw > 0 else None,
+            "r2": round(r2, 4)}
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def host_workload():
+    """Host copies of the block and its inputs (generated on the GPU when there is one)."""
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    mats = make_weights(dev)
+    xs = make_inputs(mats, N_TOKENS, dev)
+    return {n: m.cpu() for n, m in mats.items()}, {n: v.cpu() for n, v in xs.items()}
+
+
+class OracleRunner:
+    """The oracle as it stands, on host copies of the same block (replica 0)."""
+
+    def __init__(self, mats, xs):
+        import oracle
+        self.o = oracle
+        self.xs = {n: v.numpy() for n, v in xs.items()}
+        self.pools = {}
+        for name, d_out, d_in, _ in SITES:
+            wb = mats[name].view(torch.int16).numpy().view(np.uint16)
+            self.pools[name] = oracle.pack(wb, oracle.FULL_BF16)
+
+    def token(self, t):
+        o = self.o
+        for name, d_out, d_in, _ in SITES:
+            kf, ka = k_counts(d_in)
+            st, tier, fi, ai, c = o.tiers(self.xs[name][t], o.MODE_TOPK, k_full=kf, k_approx=ka)
+            o.tiered_gemv(*self.pools[name], o.FULL_BF16, d_out, d_in, self.xs[name][t], tier)
+
+
+def cpu_baseline(n_tokens, mats, xs):
+    r = OracleRunner(mats, xs)
+    t0 = time.perf_counter()
+    for t in range(n_tokens):
+        r.token(t)
+    dt = time.perf_counter() - t0
+    return {"value": round(dt * 1e6 / n_tokens, 1), "unit": "us/token/layer", "cores": 1,
+            "kind": "oracle",
+            "sample": f"{n_tokens} of the {N_TOKENS} tokens, all four sites, single-threaded C "
+                      f"oracle (fp64), {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    r = OracleRunner(*host_workload())
+    per_step = max(1, args.ref_tokens)
+    for w in range(args.warmup):
+        r.token(w % N_TOKENS)
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        for k in range(per_step):
+            r.token((s * per_step + k) % N_TOKENS)
+    dt = time.perf_counter() - t0
+    val = dt * 1e6 / (args.steps * per_step)
+    line = {"metric": METRIC, "value": round(val, 1), "unit": "us/token/layer", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt * 1e3 / args.steps, 3), "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": WORKLOAD, "tokens_per_step": per_step,
+                       "tiers": {"skip": SKIP, "approx": APPROX, "full": FULL}},
+            "cpu_baseline": {"value": round(val, 1), "unit": "us/token/layer", "cores": 1,
+                             "kind": "oracle",
+                             "sample": f"{per_step} token(s) per step, all four sites"},
+            "e2e": {"value": round(val, 1), "unit": "us/token/layer", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["spax", "reference"], default="spax")
+    ap.add_argument("--tokens", type=int, default=N_TOKENS)
+    ap.add_argument("--replicas", type=int, default=N_REPLICAS)
+    ap.add_argument("--cpu-tokens", type=int, default=24)
+    ap.add_argument("--ref-tokens", type=int, default=1)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank, world, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            return run_reference(args, rank, world)
+        res, sites, tot_bytes, tot_ms, lps, h2d, d2h, clocks, host = run_gpu(args, rank, world, local)
+        ms = res["tiered"]
+        value = us_per_token_layer(ms, args.tokens, world)
+        dense = us_per_token_layer(res["dense"], args.tokens, world)
+        e2e = us_per_token_layer(res["e2e"], args.tokens, world)
+        peak, peak_kind = measured_peak()
+        achieved = tot_bytes / (tot_ms * 1e-3) / 1e9
+        step_bytes = sum(s["bytes_per_launch"] for s in sites.values()) * args.tokens
+        dense_bytes = sum(2 * d_out * d_in for _, d_out, d_in, _ in SITES) * args.tokens
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": "us/token/layer",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 4), "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32-accumulate (bf16 + 2-bit weights)",
+            "data": "synthetic (seeded bf16 N(0,0.02) weights, Laplace(0,1) activations)",
+            "config": {"workload": WORKLOAD, "tokens_per_step": args.tokens,
+                       "tiers": {"skip": SKIP, "approx": APPROX, "full": FULL, "rule": "topk"},
+                       "weight_replicas": args.replicas,
+                       "l2": "inputs larger than L2: each token reads one of the weight replicas",
+                       "parallelism": f"replicas x{world}"},
+            "effective_GBps": round(step_bytes / (ms * 1e-3) / 1e9, 1),
+            "frac_of_8TBps": round(step_bytes / (ms * 1e-3) / 8e12, 4),
+            "dense_us_per_token_layer": round(dense, 3),
+            "dense_effective_GBps": round(dense_bytes / (res["dense"] * 1e-3) / 1e9, 1),
+            "speedup_vs_dense": round(dense / value, 3),
+            "sites": sites,
+            "fit_time_vs_bytes": {"tiered": fit_c0_bw([(v["bytes_per_launch"], v["gemv_us"]) for v in sites.values()]),
+                                  "dense": fit_c0_bw([(2 * v["d_out"] * v["d_in"], v["dense_us"]) for v in sites.values()])},
+            "roofline": {"bound": "hbm", "kernel": "tiered_gemv_kernel",
+                         "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "peak_source": peak_kind,
+                         "traffic": None},
+            "e2e": {"value": round(e2e, 3), "unit": "us/token/layer", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": lps * args.steps,
+            "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+        }
+        if host is not None:
+            line["cpu_baseline"] = cpu_baseline(args.cpu_tokens, *host)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return 0
+    finally:
+        if dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -75,7 +75,7 @@ typedef enum { SPAX_MASK_THRESHOLD = 0, SPAX_MASK_TOPK = 1, SPAX_MASK_GUIDED = 2
 typedef enum { SPAX_OP_TIERED_GEMV = 0, SPAX_OP_DENSE_GEMV = 1, SPAX_OP_CALIBRATE = 2 } spax_op;
 
 /* Largest d_in a mask call accepts (the activation vector lives in one CTA's shared memory). */
-#define SPAX_MASK_MAX_DIN 49152
+#define SPAX_MASK_MAX_DIN 32768
 
 /*
  * Tier-rule parameters for spax_build_mask.
@@ -201,7 +201,8 @@ spax_status spax_dense_gemv(const void* d_Wt, const float* d_x, float* d_y, int 
 
 /*
  * Device workspace bytes an op needs for a shape on the CURRENT device (the split count
- * depends on its SM count). Returns 0 for an invalid op or shape.
+ * depends on its SM count), enough for either full-tier format. Returns 0 for an invalid op or
+ * shape.
  */
 size_t spax_workspace_bytes(int op, int d_out, int d_in);
 

@@ -186,7 +186,8 @@ int oracle_tiers(const float* x, int d, int mode, float t_skip, float t_full, in
 
 /*
  * 2-bit asymmetric quantiser of one 128-row group (values w[0..n) as bf16 bits), fp32:
- *   mn, mx = min, max; min_b = bf16(mn) (exact, mn is a bf16 value); scale_b = bf16_rne((mx-mn)/3);
+ *   mn, mx = min, max (a zero extreme counts as +0); min_b = bf16(mn) (exact, mn is a bf16
+ *   value); scale_b = bf16_rne((mx-mn)/3);
  *   q = clamp(rint_even((w - min_b) / scale_b), 0, 3), or 0 when scale_b == 0.
  * Dequantised value: min_b + q * scale_b.
  */
@@ -198,6 +199,10 @@ void oracle_quant2_group(const uint16_t* w, int n, uint8_t* q, uint16_t* scale_b
     if (v < mn) mn = v;
     if (v > mx) mx = v;
   }
+  /* a zero extreme is taken as +0 (adding +0 maps -0 to +0 and leaves every other value) */
+  volatile float mn0 = mn + 0.0f, mx0 = mx + 0.0f;
+  mn = mn0;
+  mx = mx0;
   volatile float range = mx - mn; /* volatile: keep each fp32 step rounded on its own */
   volatile float third = range / 3.0f;
   uint16_t sb = oracle_f32_to_bf16(third);

@@ -1,0 +1,604 @@
+// gemv.cu — the fused tiered gather-GEMV (and the dense bf16 GEMV built from the same kernel).
+//
+// y = Σ_{j in full} x_j W[:,j] + Σ_{j in approx} x_j (min_g + q·scale_g)[:,j]   (fp32 accumulate)
+//
+// Sources: SpAx (arXiv 2610.02598), Abstract — original weights for the largest |x|,
+// approximate weights for smaller |x|, nothing for the rest; eigenradar commentary on SpAx,
+// "The route outside GPU memory" — cost is bytes moved per token plus the time to reconstruct
+// the two-bit approximations on the GPU.
+//
+// Design (B200, HBM-bound; no tensor cores — a batch-one GEMV has no reuse):
+//   * Grid = T row tiles (R = 512*RG rows) x S column splits, one CTA of 16 warps per SM (single
+//     wave). Split s takes positions s, s+S, s+2S, ... of the compacted approx list and of the
+//     full list, so every CTA gets the same mix of byte-heavy (bf16/int4) and ALU-heavy (2-bit)
+//     columns and the S CTAs of a tile sweep neighbouring columns together. The positions do not
+//     depend on the counts, so the index loads are issued together with the device-side counts
+//     load (one memory round trip, no host sync).
+//   * Warp (rg, cg) owns rows [512 rg, 512 rg + 512) of the tile and every CG-th column of the
+//     CTA's share. Lane l owns rows 8l..8l+7 and 256+8l..256+8l+7 in all three formats, so bf16,
+//     int4 and 2-bit contributions land in the same 16 fp32 accumulators. Weights stream straight
+//     into registers with 16-byte loads marked evict-first, U bf16 columns in flight per warp;
+//     the small 2-bit and int4 records are staged per warp in shared memory, a batch of 16-32
+//     columns at a time. (Measured on B200: one-warp-issued 1-D bulk copies of 0.1-4 KB column
+//     segments are issue-bound at 0.5-3 TB/s; plain 16-byte loads from many warps reach
+//     6.4-6.9 TB/s.)
+//   * 2-bit and int4 codes become floats with one LOP3 each: the code is masked into the
+//     mantissa of a power-of-two constant C (value C + q exactly), multiplied by x_j*scale and
+//     the constant's contribution C*Σ x_j*scale is removed once per row at the end.
+//   * Warps' partial rows are combined in shared memory in a fixed order; split-K partials go to
+//     a workspace and the last CTA of each tile to arrive (arrival ticket: no CTA ever waits for
+//     another) sums the S partials in split order, so results are bit-reproducible.
+#include "common.cuh"
+#include "internal.h"
+
+namespace spax {
+
+constexpr int kGemvWarps = 16;
+constexpr int kGemvThreads = kGemvWarps * 32;
+constexpr int kGemvMeta = 1024;  // metadata slots per list per chunk
+constexpr int kGemvU = 4;        // columns in flight per warp
+
+// Small records (2-bit: 144 B per column and 512 rows; int4: 272 B per column and 512 rows) are
+// fetched a batch of 16 at a time into a per-warp staging buffer with coalesced 16-byte loads,
+// so a warp keeps 2-4 KB in flight instead of a few bytes per lane.
+constexpr int kBatch2 = 16;                // 2-bit columns per staged batch
+constexpr int kBatch4 = 16;                // int4 columns per staged batch
+constexpr int kStageRecBytes = 16 * 272;   // = max(16 * 144, 16 * 272)
+constexpr int kStageWarpBytes = kStageRecBytes + 16 * 16;  // + 4 coefficients per column
+
+template <int RG>
+struct GemvCfg {
+  static constexpr int R = 512 * RG;          // rows per tile
+  static constexpr int CG = kGemvWarps / RG;  // column groups
+  static constexpr int kSlotFloats = (R / 32) * 36;  // combine slot: 36 floats per 32 rows
+  static constexpr size_t kSmemBytes = size_t(2) * kGemvMeta * 4 + size_t(CG) * kSlotFloats * 4 +
+                                       size_t(kGemvWarps) * kStageWarpBytes;
+  static_assert(CG >= 4, "reduction scratch must fit the combine area");
+  static_assert(kBatch4 * 272 <= kStageRecBytes && kBatch2 * 144 <= kStageRecBytes, "staging");
+};
+
+struct GemvParams {
+  const uint8_t* full;
+  const uint8_t* approx;
+  const float* x;
+  const int32_t* fidx;
+  const int32_t* aidx;
+  const int32_t* counts;
+  float* y;
+  float* part;      // [S][d_out]
+  float* gpart;     // [NG][d_out]
+  uint32_t* gtick;  // [T][NG]
+  uint32_t* ttick;  // [T]
+  int32_t* status;
+  long long full_col_stride;    // bytes between full-pool columns
+  long long approx_col_stride;  // bytes between approx-pool columns
+  int d_out, d_in, S, G, NG;
+};
+
+// Code -> float: (word & (mask << p)) | bits(C) is the float C + code, exactly, when C = 2^(23-p)
+// (the code lands in the mantissa bits whose weight is 1).
+__device__ __forceinline__ float code_f(uint32_t rot, uint32_t mask_at_p, uint32_t c_bits) {
+  return __uint_as_float((rot & mask_at_p) | c_bits);
+}
+
+// Index of row r inside a combine slot (36 floats per 32 rows: padding spreads the banks).
+__device__ __forceinline__ int red_row(int r) { return (r >> 5) * 36 + (r & 31); }
+
+__device__ __forceinline__ uint4 ld_stream128(const uint8_t* p) {
+  return __ldcs(reinterpret_cast<const uint4*>(p));
+}
+__device__ __forceinline__ uint32_t ld_stream32(const uint8_t* p) {
+  return __ldcs(reinterpret_cast<const unsigned int*>(p));
+}
+__device__ __forceinline__ uint32_t ld_stream16(const uint8_t* p) {
+  return __ldcs(reinterpret_cast<const unsigned short*>(p));
+}
+
+// Fixed-order sum of `cnt` partial rows [r0, r0+rows) (row stride d_out), written to dst + r0.
+// The partials are cut into consecutive batches of kBatch, each summed by one thread with all
+// its loads in flight; the batch sums are then added in batch order. The association depends only
+// on cnt, so the result is reproducible.
+template <int NT>
+__device__ void reduce_rows(const float* src, int cnt, int d_out, int r0, int rows, float* dst,
+                            int tid, float4* scratch /* [nbatch][rows/4] */) {
+  constexpr int kBatch = 16;
+  const int n4 = rows >> 2;
+  const int nb = (cnt + kBatch - 1) / kBatch;  // <= 3 when cnt <= 48
+  const size_t stride4 = static_cast<size_t>(d_out) >> 2;
+  const float4* s4 = reinterpret_cast<const float4*>(src + r0);
+  for (int item = tid; item < n4 * nb; item += NT) {
+    const int i = item % n4, b = item / n4;
+    const int k0 = b * kBatch, kn = min(cnt - k0, kBatch);
+    float4 v[kBatch];
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k)
+      if (k < kn) v[k] = __ldcg(s4 + (size_t)(k0 + k) * stride4 + i);
+    float4 acc = v[0];
+#pragma unroll
+    for (int k = 1; k < kBatch; ++k)
+      if (k < kn) {
+        acc.x += v[k].x;
+        acc.y += v[k].y;
+        acc.z += v[k].z;
+        acc.w += v[k].w;
+      }
+    if (nb == 1)
+      reinterpret_cast<float4*>(dst + r0)[i] = acc;
+    else
+      scratch[b * n4 + i] = acc;
+  }
+  if (nb == 1) return;
+  __syncthreads();
+  for (int i = tid; i < n4; i += NT) {
+    float4 acc = scratch[i];
+    for (int b = 1; b < nb; ++b) {
+      const float4 v = scratch[b * n4 + i];
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    reinterpret_cast<float4*>(dst + r0)[i] = acc;
+  }
+}
+
+template <int RG, int FMT, bool DENSE>
+__global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const GemvParams p) {
+  using C = GemvCfg<RG>;
+  constexpr int R = C::R, CG = C::CG, U = kGemvU;
+  static_assert(FMT == SPAX_FULL_BF16 || !DENSE, "the dense GEMV reads the bf16 pool");
+  extern __shared__ __align__(128) uint8_t smem[];
+  int32_t* meta_col_a = reinterpret_cast<int32_t*>(smem);
+  int32_t* meta_col_f = meta_col_a + kGemvMeta;
+  float* red = reinterpret_cast<float*>(meta_col_f + kGemvMeta);  // [CG][kSlotFloats]
+  __shared__ int s_bad, s_last;
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int tile = blockIdx.x, split = blockIdx.y, S = p.S;
+  const int r0 = tile * R;
+  const int rows_here = min(R, p.d_out - r0);
+  const int rg = warp / CG, cg = warp % CG;
+  const int rb = r0 + 512 * rg;              // first row of this warp
+  const bool wrows = rb < p.d_out;           // the warp has rows (ragged last tile)
+  const bool v0 = rb + 8 * lane < p.d_out;   // lane's first 8-row chunk is inside the matrix
+  const bool v1 = rb + 256 + 8 * lane < p.d_out;
+  // per-warp staging buffer: kBatch records, then their coefficients x*scale per 128-row group
+  uint8_t* stage = reinterpret_cast<uint8_t*>(red + CG * C::kSlotFloats) + warp * kStageWarpBytes;
+  const uint32_t stage_s = smem_u32(stage);
+  const uint32_t coef_s = stage_s + kStageRecBytes;
+
+  if (tid == 0) {
+    s_bad = 0;
+    s_last = 0;
+  }
+  pdl_wait();
+  pdl_launch_dependents();
+
+  // ---- counts and (speculatively) this split's first kGemvMeta positions of both lists ----
+  int Kf, Ka;
+  if (DENSE) {
+    Kf = p.d_in;
+    Ka = 0;
+  } else {
+    Kf = __ldcg(p.counts);
+    Ka = __ldcg(p.counts + 1);
+    for (int i = tid; i < kGemvMeta; i += kGemvThreads) {
+      const long long pos = split + (long long)S * i;
+      if (pos < p.d_in) {
+        meta_col_a[i] = __ldcg(p.aidx + pos);
+        meta_col_f[i] = __ldcg(p.fidx + pos);
+      }
+    }
+    if (Kf < 0 || Ka < 0 || Kf > p.d_in || Ka > p.d_in - Kf) {
+      if (tid == 0) record_status(p.status, SPAX_ERR_INDEX);
+      Kf = 0;
+      Ka = 0;
+    }
+  }
+  const int nf = Kf > split ? (Kf - split + S - 1) / S : 0;  // items of this split
+  const int na = Ka > split ? (Ka - split + S - 1) / S : 0;
+  const int nchunks = (max(nf, na) + kGemvMeta - 1) / kGemvMeta;
+
+  // this warp's slice of the packed pools
+  const long long off_full = 2LL * (rb + 8 * lane);  // bf16 pool
+  const long long off_approx = (long long)(rb / 512) * 144;
+  const long long nib0 = (long long)(rb / 1024) * 528 + ((rb / 512) & 1) * 256;  // int4 pool
+  const long long scl0 = (long long)(rb / 1024) * 528 + 512;
+  const int half4 = (rb / 512) & 1;  // which half of its 1024-row int4 record the warp reads
+
+  f2 acc[8];  // rows 8l..8l+7 (acc[0..3]) and 256+8l..256+8l+7 (acc[4..7]), as pairs
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = f2{0.f, 0.f};
+  // per 128-row group g of the warp's 512 rows, summed over the columns this lane prepared:
+  // 2-bit Σ x*scale and Σ x*min, int4 Σ x*scale (reduced over the warp at the end)
+  float sA[4] = {0.f, 0.f, 0.f, 0.f}, bA[4] = {0.f, 0.f, 0.f, 0.f}, s4[4] = {0.f, 0.f, 0.f, 0.f};
+
+  // Stage nb (<= kBatch2) 2-bit records of columns meta_col_a[cg + CG*(k0 + k)] and prepare
+  // their coefficients c[k][g] = x*scale_g (lane k), accumulating the group sums.
+  auto stage_approx = [&](int k0, int nb) {
+    __syncwarp();
+    constexpr int kChunks2 = (kBatch2 * 9 + 31) / 32;  // 16-byte chunks per lane
+    uint4 v[kChunks2];
+#pragma unroll
+    for (int t = 0; t < kChunks2; ++t) {
+      const int q = t * 32 + lane, k = q / 9, piece = q - 9 * k;
+      const int col = k < nb ? max(meta_col_a[cg + CG * (k0 + k)], 0) : 0;
+      v[t] = k < nb ? ld_stream128(p.approx + col * p.approx_col_stride + off_approx + 16 * piece)
+                    : make_uint4(0u, 0u, 0u, 0u);
+    }
+    float xk = 0.f;
+    if (lane < nb) {
+      const int col = meta_col_a[cg + CG * (k0 + lane)];
+      xk = col >= 0 ? __ldg(p.x + col) : 0.f;  // an invalid column contributes zero
+    }
+#pragma unroll
+    for (int t = 0; t < kChunks2; ++t)
+      if (t * 32 + lane < kBatch2 * 9) reinterpret_cast<uint4*>(stage)[t * 32 + lane] = v[t];
+    __syncwarp();
+    if (lane < nb) {
+      const uint4 sm = lds128(stage_s + 144 * lane + 128);  // (scale | min << 16) per group
+      const uint32_t w[4] = {sm.x, sm.y, sm.z, sm.w};
+      float c[4];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        c[g] = xk * __uint_as_float(w[g] << 16);
+        sA[g] += c[g];
+        bA[g] = fmaf(xk, __uint_as_float(w[g] & 0xFFFF0000u), bA[g]);
+      }
+      asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(coef_s + 16 * lane), "f"(c[0]),
+                   "f"(c[1]), "f"(c[2]), "f"(c[3]));
+    }
+    __syncwarp();
+  };
+
+  // 2-bit column k of the staged batch: 16 rows per word, row k at bits 2k. Rotations by 17 and
+  // 25 bring rows 0-3 and 4-7 of an 8-row group to mantissa bits 15, 17, 19, 21: values 256+q,
+  // 64+q, 16+q, 4+q.
+  auto decode_approx = [&](int k) {
+    const uint32_t rec = stage_s + 144 * k;
+    const uint32_t q01 = lds32(rec + 2 * (lane & ~1)) >> (16 * (lane & 1));  // 2 bytes at 2*lane
+    const uint32_t q11 = lds32(rec + 64 + 2 * (lane & ~1)) >> (16 * (lane & 1));
+    const float c0 = __uint_as_float(lds32(coef_s + 16 * k + 4 * (lane / 16)));
+    const float c1 = __uint_as_float(lds32(coef_s + 16 * k + 4 * (2 + lane / 16)));
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      const uint32_t w = b ? q11 : q01;
+      const f2 c2 = b ? f2{c1, c1} : f2{c0, c0};
+      const uint32_t ra = __funnelshift_r(w, w, 17), rc = __funnelshift_r(w, w, 25);
+      acc[4 * b + 0] = ffma2(f2{code_f(ra, 3u << 15, 0x43800000u), code_f(ra, 3u << 17, 0x42800000u)}, c2, acc[4 * b + 0]);
+      acc[4 * b + 1] = ffma2(f2{code_f(ra, 3u << 19, 0x41800000u), code_f(ra, 3u << 21, 0x40800000u)}, c2, acc[4 * b + 1]);
+      acc[4 * b + 2] = ffma2(f2{code_f(rc, 3u << 15, 0x43800000u), code_f(rc, 3u << 17, 0x42800000u)}, c2, acc[4 * b + 2]);
+      acc[4 * b + 3] = ffma2(f2{code_f(rc, 3u << 19, 0x41800000u), code_f(rc, 3u << 21, 0x40800000u)}, c2, acc[4 * b + 3]);
+    }
+  };
+
+  for (int ch = 0; ch < nchunks; ++ch) {
+    const int ib0 = ch * kGemvMeta;
+    const int nac = max(0, min(na - ib0, kGemvMeta));
+    const int nfc = max(0, min(nf - ib0, kGemvMeta));
+    if (ch > 0) {
+      __syncthreads();  // every warp is done with the previous chunk's metadata
+      if (!DENSE) {
+        for (int i = tid; i < kGemvMeta; i += kGemvThreads) {
+          const long long pos = split + (long long)S * (ib0 + i);
+          if (i < nac) meta_col_a[i] = __ldcg(p.aidx + pos);
+          if (i < nfc) meta_col_f[i] = __ldcg(p.fidx + pos);
+        }
+      }
+    }
+    // validate this chunk's columns (the dense GEMV generates them); an invalid one becomes -1
+    for (int i = tid; i < kGemvMeta; i += kGemvThreads) {
+      if (i < nac && (unsigned)meta_col_a[i] >= (unsigned)p.d_in) {
+        s_bad = 1;
+        meta_col_a[i] = -1;
+      }
+      if (DENSE) {
+        if (i < nfc) meta_col_f[i] = split + S * (ib0 + i);
+      } else if (i < nfc && (unsigned)meta_col_f[i] >= (unsigned)p.d_in) {
+        s_bad = 1;
+        meta_col_f[i] = -1;
+      }
+    }
+    __syncthreads();
+    if (!wrows) continue;
+    const int nAw = nac > cg ? (nac - cg + CG - 1) / CG : 0;  // this warp's 2-bit columns
+    const int nFw = nfc > cg ? (nfc - cg + CG - 1) / CG : 0;  // this warp's full columns
+
+    if constexpr (FMT == SPAX_FULL_BF16) {
+      // bf16 batches of U columns interleaved with 2-bit columns, so the dequant work of the
+      // 2-bit tier runs while the bf16 loads are in flight
+      const int per_it = nFw > 0 ? (nAw * U + nFw - 1) / nFw : nAw;
+      int ka = 0, kf = 0, sbeg = 0, send = 0;
+      while (ka < nAw || kf < nFw) {
+        const int nfb = max(0, min(U, nFw - kf));
+        uint4 w0[U], w1[U];
+        float xf[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          int col = u < nfb ? meta_col_f[cg + CG * (kf + u)] : -1;
+          xf[u] = col >= 0 ? __ldg(p.x + col) : 0.f;
+          const uint8_t* src = p.full + max(col, 0) * p.full_col_stride + off_full;
+          w0[u] = (u < nfb && v0) ? ld_stream128(src) : make_uint4(0u, 0u, 0u, 0u);
+          w1[u] = (u < nfb && v1) ? ld_stream128(src + 512) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        int todo = (kf + nfb < nFw) ? min(per_it, nAw - ka) : nAw - ka;
+        while (todo > 0) {
+          if (ka == send) {
+            sbeg = ka;
+            send = ka + min(kBatch2, nAw - ka);
+            stage_approx(sbeg, send - sbeg);
+          }
+          const int n = min(todo, send - ka);
+#pragma unroll 2
+          for (int k = ka; k < ka + n; ++k) decode_approx(k - sbeg);
+          ka += n;
+          todo -= n;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const f2 x2{xf[u], xf[u]};
+          acc[0] = ffma2(bf16x2_to_f2(w0[u].x), x2, acc[0]);
+          acc[1] = ffma2(bf16x2_to_f2(w0[u].y), x2, acc[1]);
+          acc[2] = ffma2(bf16x2_to_f2(w0[u].z), x2, acc[2]);
+          acc[3] = ffma2(bf16x2_to_f2(w0[u].w), x2, acc[3]);
+          acc[4] = ffma2(bf16x2_to_f2(w1[u].x), x2, acc[4]);
+          acc[5] = ffma2(bf16x2_to_f2(w1[u].y), x2, acc[5]);
+          acc[6] = ffma2(bf16x2_to_f2(w1[u].z), x2, acc[6]);
+          acc[7] = ffma2(bf16x2_to_f2(w1[u].w), x2, acc[7]);
+        }
+        kf += nfb;
+      }
+    } else {
+      for (int ka = 0; ka < nAw; ka += kBatch2) {
+        const int nb = min(kBatch2, nAw - ka);
+        stage_approx(ka, nb);
+#pragma unroll 2
+        for (int k = 0; k < nb; ++k) decode_approx(k);
+      }
+      // int4: 8 rows per word, nibble of row k at bits 4k, stored as u = q + 8. Rotations by
+      // 17, 25, 1, 9 bring rows (0,1), (2,3), (4,5), (6,7) to mantissa bits 15 and 19:
+      // values 256 + u and 16 + u. A staged half-record is the warp's 256 bytes of nibbles
+      // followed by the record's 16 bytes of scales (17 chunks of 16 B).
+      for (int kf = 0; kf < nFw; kf += kBatch4) {
+        const int nb = min(kBatch4, nFw - kf);
+        __syncwarp();
+        uint4 v[9];
+#pragma unroll
+        for (int t = 0; t < 9; ++t) {
+          const int q = t * 32 + lane, k = q / 17, piece = q - 17 * k;
+          const int col = k < nb ? max(meta_col_f[cg + CG * (kf + k)], 0) : 0;
+          const uint8_t* src = p.full + col * p.full_col_stride;
+          v[t] = (q < 17 * kBatch4 && k < nb)
+                     ? ld_stream128(piece < 16 ? src + nib0 + 16 * piece : src + scl0)
+                     : make_uint4(0u, 0u, 0u, 0u);
+        }
+        float xk = 0.f;
+        if (lane < nb) {
+          const int col = meta_col_f[cg + CG * (kf + lane)];
+          xk = col >= 0 ? __ldg(p.x + col) : 0.f;
+        }
+#pragma unroll
+        for (int t = 0; t < 9; ++t)
+          if (t * 32 + lane < 17 * kBatch4) reinterpret_cast<uint4*>(stage)[t * 32 + lane] = v[t];
+        __syncwarp();
+        if (lane < nb) {
+          // this half's four group scales: bf16 scales [4*half4, 4*half4 + 4) of the record
+          const uint2 sw = lds64(stage_s + 272 * lane + 256 + 8 * half4);
+          const uint32_t w[4] = {sw.x << 16, sw.x & 0xFFFF0000u, sw.y << 16, sw.y & 0xFFFF0000u};
+          float c[4];
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            c[g] = xk * __uint_as_float(w[g]);
+            s4[g] += c[g];
+          }
+          asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(coef_s + 16 * lane),
+                       "f"(c[0]), "f"(c[1]), "f"(c[2]), "f"(c[3]));
+        }
+        __syncwarp();
+#pragma unroll 2
+        for (int k = 0; k < nb; ++k) {
+          const uint32_t rec = stage_s + 272 * k;
+          const uint32_t n0 = lds32(rec + 4 * lane), n1 = lds32(rec + 128 + 4 * lane);
+          const float c0 = __uint_as_float(lds32(coef_s + 16 * k + 4 * (lane / 16)));
+          const float c1 = __uint_as_float(lds32(coef_s + 16 * k + 4 * (2 + lane / 16)));
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            const uint32_t w = b ? n1 : n0;
+            const f2 c2 = b ? f2{c1, c1} : f2{c0, c0};
+            const uint32_t rA = __funnelshift_r(w, w, 17), rB = __funnelshift_r(w, w, 25);
+            const uint32_t rC = __funnelshift_r(w, w, 1), rD = __funnelshift_r(w, w, 9);
+            acc[4 * b + 0] = ffma2(f2{code_f(rA, 0xFu << 15, 0x43800000u), code_f(rA, 0xFu << 19, 0x41800000u)}, c2, acc[4 * b + 0]);
+            acc[4 * b + 1] = ffma2(f2{code_f(rB, 0xFu << 15, 0x43800000u), code_f(rB, 0xFu << 19, 0x41800000u)}, c2, acc[4 * b + 1]);
+            acc[4 * b + 2] = ffma2(f2{code_f(rC, 0xFu << 15, 0x43800000u), code_f(rC, 0xFu << 19, 0x41800000u)}, c2, acc[4 * b + 2]);
+            acc[4 * b + 3] = ffma2(f2{code_f(rD, 0xFu << 15, 0x43800000u), code_f(rD, 0xFu << 19, 0x41800000u)}, c2, acc[4 * b + 3]);
+          }
+        }
+      }
+    }
+  }
+  if (tid == 0 && s_bad) record_status(p.status, SPAX_ERR_INDEX);
+
+  // warp totals of the per-group sums (xor butterfly: every lane ends with the same totals)
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      if constexpr (!DENSE) {
+        sA[g] += __shfl_xor_sync(0xffffffffu, sA[g], o);
+        bA[g] += __shfl_xor_sync(0xffffffffu, bA[g], o);
+      }
+      if constexpr (FMT == SPAX_FULL_INT4_G128) s4[g] += __shfl_xor_sync(0xffffffffu, s4[g], o);
+    }
+  }
+  const int g0 = lane / 16;  // group of the lane's first 8 rows; the second chunk is group g0 + 2
+  const float sumA0 = g0 ? sA[1] : sA[0], sumA1 = g0 ? sA[3] : sA[2];
+  const float baseA0 = g0 ? bA[1] : bA[0], baseA1 = g0 ? bA[3] : bA[2];
+  const float sum40 = g0 ? s4[1] : s4[0], sum41 = g0 ? s4[3] : s4[2];
+
+  // ---- combine the warps' partial rows inside the CTA (fixed order) ----
+  if (wrows) {
+    // remove the mantissa constants: 2-bit rows 4i+{0,1,2,3} carry {256,64,16,4}*Σc, int4 even
+    // rows (256+8)*Σc and odd rows (16+8)*Σc; add Σ x*min for the 2-bit tier
+    float* slot = red + cg * C::kSlotFloats;
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      const float sa = b ? sumA1 : sumA0, ba = b ? baseA1 : baseA0, s4 = b ? sum41 : sum40;
+      const float k0 = ba - 256.f * sa, k1 = ba - 64.f * sa, k2 = ba - 16.f * sa, k3 = ba - 4.f * sa;
+      const float e = -264.f * s4, o = -24.f * s4;
+      float4 lo, hi;
+      lo.x = acc[4 * b + 0].x + k0 + e;
+      lo.y = acc[4 * b + 0].y + k1 + o;
+      lo.z = acc[4 * b + 1].x + k2 + e;
+      lo.w = acc[4 * b + 1].y + k3 + o;
+      hi.x = acc[4 * b + 2].x + k0 + e;
+      hi.y = acc[4 * b + 2].y + k1 + o;
+      hi.z = acc[4 * b + 3].x + k2 + e;
+      hi.w = acc[4 * b + 3].y + k3 + o;
+      float* dst = slot + red_row(512 * rg + 256 * b + 8 * lane);
+      reinterpret_cast<float4*>(dst)[0] = lo;
+      reinterpret_cast<float4*>(dst)[1] = hi;
+    }
+  }
+  __syncthreads();
+
+  float* out_base = (S == 1) ? p.y : p.part + (size_t)split * p.d_out;
+  for (int i = tid; i < rows_here / 4; i += kGemvThreads) {
+    float4 v = reinterpret_cast<const float4*>(red + red_row(4 * i))[0];
+#pragma unroll
+    for (int c = 1; c < CG; ++c) {
+      const float4 w = reinterpret_cast<const float4*>(red + c * C::kSlotFloats + red_row(4 * i))[0];
+      v.x += w.x;
+      v.y += w.y;
+      v.z += w.z;
+      v.w += w.w;
+    }
+    reinterpret_cast<float4*>(out_base + r0)[i] = v;
+  }
+  if (S == 1) return;
+
+  // ---- split-K: the last split of each group (then of the tile) to arrive sums in order ----
+  const int grp = split / p.G;
+  const int gbeg = grp * p.G;
+  const int gsz = min(p.G, S - gbeg);
+  float4* scratch = reinterpret_cast<float4*>(red);  // [<=4][R/4] fits in CG >= 4 slots
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t* t = p.gtick + (size_t)tile * p.NG + grp;
+    const uint32_t old = atomicAdd(t, 1u);
+    const int last = (old == (uint32_t)(gsz - 1));
+    if (last) *t = 0u;  // every other split of the group has arrived: reset for the next call
+    s_last = last;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  float* gdst = (p.NG == 1) ? p.y : p.gpart + (size_t)grp * p.d_out;
+  reduce_rows<kGemvThreads>(p.part + (size_t)gbeg * p.d_out, gsz, p.d_out, r0, rows_here, gdst,
+                            tid, scratch);
+  if (p.NG == 1) return;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t* t = p.ttick + tile;
+    const uint32_t old = atomicAdd(t, 1u);
+    const int last = (old == (uint32_t)(p.NG - 1));
+    if (last) *t = 0u;
+    s_last = last;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  reduce_rows<kGemvThreads>(p.gpart, p.NG, p.d_out, r0, rows_here, p.y, tid, scratch);
+}
+
+// ------------------------------------------------------------------------------------------------
+
+bool make_gemv_plan(int d_out, int d_in, int full_fmt, int sm_count, GemvPlan* plan) {
+  if (d_out < 128 || d_out % 128 != 0 || d_in < 1 || sm_count < 1) return false;
+  if (full_fmt != SPAX_FULL_BF16 && full_fmt != SPAX_FULL_INT4_G128) return false;
+  GemvPlan pl;
+  // Smallest row tile that still leaves >= 8 splits per tile: the last CTA of a tile sums
+  // S x R partial values, so a small S*R keeps the reduction short.
+  pl.R = 2048;
+  for (int r = 512; r <= 1024; r *= 2) {
+    if ((d_out + r - 1) / r <= sm_count / 8) {
+      pl.R = r;
+      break;
+    }
+  }
+  pl.T = (d_out + pl.R - 1) / pl.R;
+  pl.S = sm_count / pl.T;
+  if (pl.S < 1) pl.S = 1;
+  if (pl.S > d_in) pl.S = d_in;
+  if (pl.S > 1024) pl.S = 1024;  // keeps the reduction batches within the combine area
+  // one level (the last of the S splits sums them all) unless S is large
+  if (pl.S <= 48) {
+    pl.G = pl.S;
+  } else {
+    int g = 1;
+    while (g * g < pl.S) ++g;
+    pl.G = g;
+  }
+  pl.NG = (pl.S + pl.G - 1) / pl.G;
+  auto al = [](size_t v) { return (v + 255) & ~size_t(255); };
+  size_t off = 0;
+  pl.off_part = off;
+  off += al(size_t(pl.S) * d_out * 4);
+  pl.off_gpart = off;
+  off += al(size_t(pl.NG > 1 ? pl.NG : 0) * d_out * 4);
+  pl.off_gtick = off;
+  off += al(size_t(pl.T) * pl.NG * 4);
+  pl.off_ttick = off;
+  off += al(size_t(pl.T) * 4);
+  pl.ws_bytes = off;
+  *plan = pl;
+  return true;
+}
+
+template <int RG, int FMT, bool DENSE>
+static cudaError_t launch_one(const GemvParams& gp, const GemvPlan& pl, cudaStream_t stream) {
+  using C = GemvCfg<RG>;
+  auto kern = tiered_gemv_kernel<RG, FMT, DENSE>;
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), (int)C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3(pl.T, pl.S), dim3(kGemvThreads), C::kSmemBytes, stream, gp);
+}
+
+template <int FMT, bool DENSE>
+static cudaError_t launch_r(const GemvParams& gp, const GemvPlan& pl, cudaStream_t stream) {
+  if (pl.R == 512) return launch_one<1, FMT, DENSE>(gp, pl, stream);
+  if (pl.R == 1024) return launch_one<2, FMT, DENSE>(gp, pl, stream);
+  return launch_one<4, FMT, DENSE>(gp, pl, stream);
+}
+
+cudaError_t launch_gemv(const GemvLaunch& a, const GemvPlan& pl, cudaStream_t stream) {
+  GemvParams gp;
+  uint8_t* ws = static_cast<uint8_t*>(a.ws);
+  gp.full = static_cast<const uint8_t*>(a.full);
+  gp.approx = static_cast<const uint8_t*>(a.approx);
+  gp.x = a.x;
+  gp.fidx = a.full_idx;
+  gp.aidx = a.approx_idx;
+  gp.counts = a.counts;
+  gp.y = a.y;
+  gp.part = reinterpret_cast<float*>(ws + pl.off_part);
+  gp.gpart = reinterpret_cast<float*>(ws + pl.off_gpart);
+  gp.gtick = reinterpret_cast<uint32_t*>(ws + pl.off_gtick);
+  gp.ttick = reinterpret_cast<uint32_t*>(ws + pl.off_ttick);
+  gp.status = a.status;
+  gp.full_col_stride = a.full_fmt == SPAX_FULL_BF16 ? 2LL * a.d_out
+                                                    : (long long)((a.d_out + 1023) / 1024) * 528;
+  gp.approx_col_stride = (long long)((a.d_out + 511) / 512) * 144;
+  gp.d_out = a.d_out;
+  gp.d_in = a.d_in;
+  gp.S = pl.S;
+  gp.G = pl.G;
+  gp.NG = pl.NG;
+  if (a.dense) return launch_r<SPAX_FULL_BF16, true>(gp, pl, stream);
+  if (a.full_fmt == SPAX_FULL_BF16) return launch_r<SPAX_FULL_BF16, false>(gp, pl, stream);
+  return launch_r<SPAX_FULL_INT4_G128, false>(gp, pl, stream);
+}
+
+}  // namespace spax

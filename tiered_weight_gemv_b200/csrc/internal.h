@@ -1,0 +1,69 @@
+// internal.h — host-side declarations shared by the libspax translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/spax.h"
+
+namespace spax {
+
+// Split-K plan of one GEMV launch: grid (T row tiles) x (S column splits); the S partial sums of
+// a tile are reduced in groups of G consecutive splits (NG groups), then over the groups.
+struct GemvPlan {
+  int R, T, S, G, NG;
+  size_t off_part, off_gpart, off_gtick, off_ttick, ws_bytes;
+};
+
+int sm_count_current_device();  // cached per device; 0 on error
+bool make_gemv_plan(int d_out, int d_in, int full_fmt, int sm_count, GemvPlan* plan);
+
+struct GemvLaunch {
+  const void* full;
+  const void* approx;
+  const float* x;
+  const int32_t* full_idx;
+  const int32_t* approx_idx;
+  const int32_t* counts;
+  float* y;
+  int32_t* status;
+  void* ws;
+  int d_out, d_in, full_fmt;
+  bool dense;
+};
+cudaError_t launch_gemv(const GemvLaunch& a, const GemvPlan& plan, cudaStream_t stream);
+
+cudaError_t launch_mask(const float* x, int d_in, const spax_mask_params& p, uint8_t* tier,
+                        int32_t* full_idx, int32_t* approx_idx, int32_t* counts, int32_t* status,
+                        cudaStream_t stream);
+
+cudaError_t launch_pack(const void* W, int d_out, int d_in, int full_fmt, void* full, void* approx,
+                        cudaStream_t stream);
+
+size_t calibrate_ws_bytes();
+cudaError_t launch_calibrate(const float* X, long long M, long long idx_skip, long long idx_full,
+                             float* t_out, int32_t* status, void* ws, cudaStream_t stream);
+
+// Launch helper: every libspax kernel is launched as a programmatic dependent of its
+// predecessor in the stream (it calls griddepcontrol.wait before touching global memory).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+// Raise a kernel's dynamic shared-memory limit once per device.
+cudaError_t ensure_smem_limit(const void* kernel, int bytes);
+
+}  // namespace spax
