@@ -200,6 +200,31 @@ spax_status spax_dense_gemv(const void* d_Wt, const float* d_x, float* d_y, int 
                             int32_t* d_status, void* d_ws, size_t ws_bytes, void* stream);
 
 /*
+ * spax_tiered_gemv_fixed_scratch — the same computation as spax_tiered_gemv (same arguments
+ * minus the workspace, same results, same kernel), for callers that cannot allocate device
+ * memory where they call it: its split-K scratch is a fixed array compiled into the library
+ * (spax_fixed_scratch_bytes() = 4 MiB per device), so the call allocates nothing. The pages
+ * have no counterpart of this entry point; it is an interface convenience.
+ * - The first call on each device (with that device current) looks up the array's device
+ *   address and caches it; make that first call before any stream capture on that device.
+ * - Shapes whose split plan needs more than the array holds (more than 4096 arrival counters,
+ *   or partial sums beyond the rest of the 4 MiB; d_out up to about 1M rows on a 148-SM GPU)
+ *   are rejected with SPAX_ERR_WORKSPACE before anything is launched.
+ * - The array's arrival counters start at zero when the library loads and every completed
+ *   call leaves them at zero; nothing for the caller to initialise.
+ * - There is ONE array per device for the whole process: calls on the same device that can
+ *   overlap (other streams, other threads, concurrent graph branches) race on it and give
+ *   wrong results. Serialise them.
+ */
+spax_status spax_tiered_gemv_fixed_scratch(const spax_packed* h_W, const float* d_x,
+                                           const int32_t* d_full_idx, const int32_t* d_approx_idx,
+                                           const int32_t* d_counts, float* d_y, int32_t* d_status,
+                                           void* stream);
+
+/* Size in bytes of the per-device scratch array spax_tiered_gemv_fixed_scratch uses. */
+size_t spax_fixed_scratch_bytes(void);
+
+/*
  * Device workspace bytes an op needs for a shape on the CURRENT device (the split count
  * depends on its SM count), enough for either full-tier format. Returns 0 for an invalid op or
  * shape.

@@ -19,7 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libspax.so")
-SOURCES = ["api.cu", "gemv.cu", "mask.cu", "pack.cu", "calibrate.cu"]
+SOURCES = ["api.cu", "gemv.cu", "mask.cu", "pack.cu", "calibrate.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVFLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr",

@@ -1,0 +1,110 @@
+// noalloc.cu — spax_tiered_gemv_fixed_scratch: the tiered GEMV with its split-K scratch in a
+// fixed device array that is part of the library image, so the call allocates nothing and needs
+// no workspace argument.
+//
+// Who needs it: callers that cannot allocate device memory at the point of the call — code that
+// runs inside an allocator-free region of a larger runtime (for instance a custom allocator's
+// own callbacks, or a plugin of a host that owns every device allocation and hands out none),
+// and callers that must not make the allocator synchronise the device. The regular entry point
+// needs a caller-owned workspace; this one does not.
+//
+// Scratch layout (kFixedScratchBytes in total, 256-byte aligned):
+//   [0, kTicketBytes)                 arrival counters of the split-K reduction. They must be
+//                                     zero before a call; device globals start at zero when the
+//                                     library's module loads and every completed call leaves
+//                                     them at zero again. Nothing else ever writes this range,
+//                                     so shapes of different calls never disturb each other's
+//                                     counters.
+//   [kTicketBytes, kFixedScratchBytes) partial sums (no initial value needed).
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace spax {
+
+constexpr size_t kFixedScratchBytes = size_t(4) << 20;  // 4 MiB per device
+constexpr size_t kTicketBytes = size_t(16) << 10;       // 4096 counters
+
+static __device__ __align__(256) uint8_t g_fixed_scratch[kFixedScratchBytes];
+
+// Device address of g_fixed_scratch on the current device, looked up once per device (with that
+// device current) and cached; nullptr if the lookup failed.
+static uint8_t* fixed_scratch_current_device() {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static uint8_t* addr[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fixed_scratch) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return nullptr;
+    }
+    addr[dev] = static_cast<uint8_t*>(p);
+  }
+  return addr[dev];
+}
+
+}  // namespace spax
+
+using namespace spax;
+
+extern "C" {
+
+size_t spax_fixed_scratch_bytes(void) { return kFixedScratchBytes; }
+
+spax_status spax_tiered_gemv_fixed_scratch(const spax_packed* W, const float* x,
+                                           const int32_t* full_idx, const int32_t* approx_idx,
+                                           const int32_t* counts, float* y, int32_t* status,
+                                           void* stream) {
+  if (!W || !W->d_full || !W->d_approx || !x || !y || !full_idx || !approx_idx || !counts)
+    return SPAX_ERR_ARG;
+  if (W->full_fmt != SPAX_FULL_BF16 && W->full_fmt != SPAX_FULL_INT4_G128) return SPAX_ERR_ARG;
+  if (W->d_out < 128 || W->d_out % 128 != 0 || W->d_in < 1) return SPAX_ERR_SHAPE;
+  auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  if (!a16(W->d_full) || !a16(W->d_approx) || !a16(y)) return SPAX_ERR_ARG;
+  const int sms = sm_count_current_device();
+  if (sms < 1) return SPAX_ERR_CUDA;
+  GemvPlan pl;
+  if (!make_gemv_plan(W->d_out, W->d_in, W->full_fmt, sms, &pl)) return SPAX_ERR_SHAPE;
+  // Same plan, relocated: counters first (in their reserved range), partial sums after them.
+  auto al = [](size_t v) { return (v + 255) & ~size_t(255); };
+  const size_t gtick_bytes = al(size_t(pl.T) * pl.NG * 4);
+  const size_t tick_bytes = gtick_bytes + al(size_t(pl.T) * 4);
+  const size_t part_bytes = al(size_t(pl.S) * W->d_out * 4);
+  const size_t gpart_bytes = al(size_t(pl.NG > 1 ? pl.NG : 0) * W->d_out * 4);
+  if (tick_bytes > kTicketBytes || kTicketBytes + part_bytes + gpart_bytes > kFixedScratchBytes)
+    return SPAX_ERR_WORKSPACE;
+  pl.off_gtick = 0;
+  pl.off_ttick = gtick_bytes;
+  pl.off_part = kTicketBytes;
+  pl.off_gpart = kTicketBytes + part_bytes;
+  pl.ws_bytes = kTicketBytes + part_bytes + gpart_bytes;
+  uint8_t* scratch = fixed_scratch_current_device();
+  if (!scratch) return SPAX_ERR_CUDA;
+  GemvLaunch a;
+  a.full = W->d_full;
+  a.approx = W->d_approx;
+  a.x = x;
+  a.full_idx = full_idx;
+  a.approx_idx = approx_idx;
+  a.counts = counts;
+  a.y = y;
+  a.status = status;
+  a.ws = scratch;
+  a.d_out = W->d_out;
+  a.d_in = W->d_in;
+  a.full_fmt = W->full_fmt;
+  a.dense = false;
+  const cudaError_t e = launch_gemv(a, pl, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SPAX_ERR_CUDA;
+  }
+  return SPAX_OK;
+}
+
+}  // extern "C"

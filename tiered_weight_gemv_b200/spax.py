@@ -58,6 +58,9 @@ _SIGS = {
     "spax_build_mask": ([_P, _I, ctypes.POINTER(spax_mask_params), _P, _P, _P, _P, _P, _P], _I),
     "spax_tiered_gemv": ([ctypes.POINTER(spax_packed), _P, _P, _P, _P, _P, _P, _P, _Z, _P], _I),
     "spax_dense_gemv": ([_P, _P, _P, _I, _I, _P, _P, _Z, _P], _I),
+    "spax_tiered_gemv_fixed_scratch": ([ctypes.POINTER(spax_packed), _P, _P, _P, _P, _P, _P, _P],
+                                       _I),
+    "spax_fixed_scratch_bytes": ([], _Z),
     "spax_workspace_bytes": ([_I, _I, _I], _Z),
     "spax_gemv_plan": ([_I, _I, _I, _I, _P, _P], _I),
     "spax_block_budgets": ([_P, _I, ctypes.c_double, ctypes.c_double, ctypes.c_double,
@@ -211,6 +214,24 @@ def spax_tiered_gemv(W: PackedMatrix, x: torch.Tensor, full_idx: torch.Tensor,
         _dev(approx_idx, torch.int32, "approx_idx"), _dev(counts, torch.int32, "counts"),
         _dev(y, torch.float32, "y"), _dev(status, torch.int32, "status"), _dev(ws, None, "ws"),
         ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def spax_tiered_gemv_fixed_scratch(W: PackedMatrix, x: torch.Tensor, full_idx: torch.Tensor,
+                                   approx_idx: torch.Tensor, counts: torch.Tensor, y: torch.Tensor,
+                                   status: torch.Tensor, stream=None, desc=None) -> None:
+    """spax_tiered_gemv without a workspace argument: the library's own per-device scratch array
+    is used, so nothing is allocated. Calls on one device must not overlap."""
+    if x.numel() != W.d_in or y.numel() != W.d_out:
+        raise ValueError("x / y sizes do not match W")
+    d = W.desc() if desc is None else desc
+    _check("spax_tiered_gemv_fixed_scratch", _lib.spax_tiered_gemv_fixed_scratch(
+        ctypes.byref(d), _dev(x, torch.float32, "x"), _dev(full_idx, torch.int32, "full_idx"),
+        _dev(approx_idx, torch.int32, "approx_idx"), _dev(counts, torch.int32, "counts"),
+        _dev(y, torch.float32, "y"), _dev(status, torch.int32, "status"), _stream(stream)))
+
+
+def spax_fixed_scratch_bytes() -> int:
+    return int(_lib.spax_fixed_scratch_bytes())
 
 
 def spax_dense_gemv(Wt: torch.Tensor, x: torch.Tensor, y: torch.Tensor, d_out: int, d_in: int,
