@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libspax.so")
 SOURCES = ["api.cu", "gemv.cu", "mask.cu", "pack.cu", "calibrate.cu", "noalloc.cu"]
-HEADERS = ["common.cuh", "internal.h"]
+HEADERS = ["common.cuh", "internal.h", "select.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVFLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr",
            "-Xptxas", "-warn-spills"]
