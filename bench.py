@@ -44,13 +44,22 @@ HIDDEN, INTER = 4096, 11008
 N_TOKENS = 64
 SKIP, APPROX, FULL = 0.4, 0.3, 0.3
 N_REPLICAS = 32
-METRIC = "us/token per decoder layer (three-tier decode GEMV), with effective HBM GB/s vs dense GEMV"
+METRIC = "\u00b5s/token per decoder layer and effective HBM GB/s (fraction of 8 TB/s), vs dense GEMV"
 WORKLOAD = "llama2-7b-block-decode-b1"
 # (name, d_out, d_in, input stream tensor id); q/k/v and gate/up are concatenated along d_out
 SITES = [("qkv", 3 * HIDDEN, HIDDEN, 101), ("o", HIDDEN, HIDDEN, 102),
          ("gate_up", 2 * INTER, HIDDEN, 103), ("down", HIDDEN, INTER, None)]
 WEIGHT_IDS = {"q": 1, "k": 2, "v": 3, "o": 4, "gate": 5, "up": 6, "down": 7}
 FALLBACK_HBM_GBS = 6650.0
+
+
+def workload_config(tokens: int, replicas: int, world: int) -> dict:
+    """The workload description both arms print (the reference arm times a sample of it)."""
+    return {"workload": WORKLOAD, "tokens_per_step": tokens,
+            "tiers": {"skip": SKIP, "approx": APPROX, "full": FULL, "rule": "topk"},
+            "weight_replicas": replicas,
+            "l2": "inputs larger than L2: each token reads one of the weight replicas",
+            "parallelism": f"replicas x{world}"}
 
 
 def k_counts(d_in: int):
@@ -206,6 +215,7 @@ def run_gpu(args, rank, world, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     n_tok, n_rep = args.tokens, args.replicas
+    SEL = [s for s in SITES if not args.sites or s[0] in args.sites.split(",")]
     mats = make_weights(dev)
     xs = make_inputs(mats, n_tok, dev)
     host = None
@@ -214,7 +224,7 @@ def run_gpu(args, rank, world, local):
 
     # packed replicas (pack once, copy) and per-site buffers
     packed = {}
-    for name, d_out, d_in, _ in SITES:
+    for name, d_out, d_in, _ in SEL:
         pm = spax.alloc_packed(d_out, d_in, spax.FULL_BF16, device=dev)
         spax.spax_pack_weights(mats[name], spax.FULL_BF16, pm)
         reps = [pm] + [spax.PackedMatrix(d_out, d_in, spax.FULL_BF16, pm.full.clone(),
@@ -223,7 +233,7 @@ def run_gpu(args, rank, world, local):
     torch.cuda.synchronize()
     del mats
     buf = {}
-    for name, d_out, d_in, _ in SITES:
+    for name, d_out, d_in, _ in SEL:
         kf, ka = k_counts(d_in)
         buf[name] = dict(
             tier=torch.empty(n_tok, d_in, dtype=torch.uint8, device=dev),
@@ -241,7 +251,7 @@ def run_gpu(args, rank, world, local):
 
     def step_tiered(mask=True, gemv=True, sites=None):
         for t in range(n_tok):
-            for name, d_out, d_in, _ in SITES:
+            for name, d_out, d_in, _ in SEL:
                 if sites is not None and name not in sites:
                     continue
                 b = buf[name]
@@ -256,7 +266,7 @@ def run_gpu(args, rank, world, local):
 
     def step_dense(sites=None):
         for t in range(n_tok):
-            for name, d_out, d_in, _ in SITES:
+            for name, d_out, d_in, _ in SEL:
                 if sites is not None and name not in sites:
                     continue
                 b = buf[name]
@@ -269,7 +279,7 @@ def run_gpu(args, rank, world, local):
         step_tiered()  # eager run: fills the lists used by the GEMV-only graphs
         step_dense()
     torch.cuda.synchronize()
-    for name, *_ in SITES:
+    for name, *_ in SEL:
         st = int(buf[name]["status"].item())
         if st != 0:
             raise RuntimeError(f"device status {st} ({spax.status_string(st)}) at site {name}")
@@ -282,7 +292,7 @@ def run_gpu(args, rank, world, local):
 
     graphs["tiered"] = capture(step_tiered)
     graphs["dense"] = capture(step_dense)
-    for name, *_ in SITES:
+    for name, *_ in SEL:
         graphs["gemv_" + name] = capture(step_tiered, mask=False, gemv=True, sites=[name])
         graphs["mask_" + name] = capture(step_tiered, mask=True, gemv=False, sites=[name])
         graphs["dense_" + name] = capture(step_dense, sites=[name])
@@ -292,7 +302,7 @@ def run_gpu(args, rank, world, local):
     with sampler:
         res["tiered"] = max_over_ranks(time_graph(graphs["tiered"], args.steps, args.warmup, stream))
         res["dense"] = max_over_ranks(time_graph(graphs["dense"], args.steps, args.warmup, stream))
-        for name, *_ in SITES:
+        for name, *_ in SEL:
             res["gemv_" + name] = max_over_ranks(
                 time_graph(graphs["gemv_" + name], args.steps, args.warmup, stream))
             res["mask_" + name] = max_over_ranks(
@@ -325,17 +335,17 @@ def run_gpu(args, rank, world, local):
             torch.cuda.synchronize()
             barrier()
         res["e2e"] = max_over_ranks(s0.elapsed_time(s1) / args.steps)
-    for name, *_ in SITES:
+    for name, *_ in SEL:
         st = int(buf[name]["status"].item())
         if st != 0:
             raise RuntimeError(f"device status {st} after timing at site {name}")
         if not torch.isfinite(buf[name]["y"]).all():
             raise RuntimeError(f"non-finite output at site {name}")
 
-    launches_per_step = n_tok * len(SITES) * 2
+    launches_per_step = n_tok * len(SEL) * 2
     sites = {}
     tot_bytes = tot_ms = 0.0
-    for name, d_out, d_in, _ in SITES:
+    for name, d_out, d_in, _ in SEL:
         b = buf[name]
         by = algorithmic_bytes(d_out, d_in, b["kf"], b["ka"])
         ms = res["gemv_" + name]
@@ -365,6 +375,30 @@ def fit_c0_bw(points):
     r2 = 1.0 - float(((t - pred) ** 2).sum()) / ss if ss > 0 else 1.0
     return {"c0_us": round(float(c0), 3), "GBps": round(1e-3 / inv_bw, 1) if inv_bw > 0 else None,
             "r2": round(r2, 4)}
+
+
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "tiered_gemv_traffic.json")
+GEMV_SOURCES = ["gemv.cu", "common.cuh", "internal.h"]
+
+
+def gemv_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in GEMV_SOURCES:
+        with open(os.path.join(ROOT, "tiered_weight_gemv_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic():
+    """Per-site DRAM bytes (read + write) per tiered-GEMV launch from the committed ncu capture,
+    or None when the GEMV sources changed since it was taken."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+    except Exception:
+        return None
+    return t["sites"] if t.get("source_sha256") == gemv_source_hash() else None
 
 
 def measured_peak():
@@ -436,11 +470,12 @@ def run_reference(args, rank, world):
             "ms_per_step": round(dt * 1e3 / args.steps, 3), "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": WORKLOAD, "tokens_per_step": per_step,
-                       "tiers": {"skip": SKIP, "approx": APPROX, "full": FULL}},
+            "config": workload_config(args.tokens, args.replicas, world),
             "cpu_baseline": {"value": round(val, 1), "unit": "us/token/layer", "cores": 1,
                              "kind": "oracle",
-                             "sample": f"{per_step} token(s) per step, all four sites"},
+                             "sample": f"{per_step} of the {N_TOKENS} tokens per step (tokens "
+                                       f"cycled), all four sites, single-threaded C oracle "
+                                       f"(fp64), weight replica 0"},
             "e2e": {"value": round(val, 1), "unit": "us/token/layer", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -460,6 +495,8 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=24)
     ap.add_argument("--ref-tokens", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sites", default="", help="comma-separated subset of qkv,o,gate_up,down "
+                    "(profiling runs); the default runs the whole block")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -473,20 +510,22 @@ def main():
         dense = us_per_token_layer(res["dense"], args.tokens, world)
         e2e = us_per_token_layer(res["e2e"], args.tokens, world)
         peak, peak_kind = measured_peak()
+        traffic_sites = measured_traffic()
+        traffic = None
+        if traffic_sites and all(n in traffic_sites for n in sites):
+            traffic = round(sum(traffic_sites[n] for n in sites) / len(sites))
+            for n in sites:
+                sites[n]["dram_bytes_per_launch"] = traffic_sites[n]
         achieved = tot_bytes / (tot_ms * 1e-3) / 1e9
         step_bytes = sum(s["bytes_per_launch"] for s in sites.values()) * args.tokens
-        dense_bytes = sum(2 * d_out * d_in for _, d_out, d_in, _ in SITES) * args.tokens
+        dense_bytes = sum(2 * v["d_out"] * v["d_in"] for v in sites.values()) * args.tokens
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": "us/token/layer",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms, 4), "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32-accumulate (bf16 + 2-bit weights)",
             "data": "synthetic (seeded bf16 N(0,0.02) weights, Laplace(0,1) activations)",
-            "config": {"workload": WORKLOAD, "tokens_per_step": args.tokens,
-                       "tiers": {"skip": SKIP, "approx": APPROX, "full": FULL, "rule": "topk"},
-                       "weight_replicas": args.replicas,
-                       "l2": "inputs larger than L2: each token reads one of the weight replicas",
-                       "parallelism": f"replicas x{world}"},
+            "config": workload_config(args.tokens, args.replicas, world),
             "effective_GBps": round(step_bytes / (ms * 1e-3) / 1e9, 1),
             "frac_of_8TBps": round(step_bytes / (ms * 1e-3) / 8e12, 4),
             "dense_us_per_token_layer": round(dense, 3),
@@ -498,7 +537,8 @@ def main():
             "roofline": {"bound": "hbm", "kernel": "tiered_gemv_kernel",
                          "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "peak_source": peak_kind,
-                         "traffic": None},
+                         "traffic": traffic,
+                         "algorithmic_bytes_per_launch": round(tot_bytes / args.tokens / len(sites))},
             "e2e": {"value": round(e2e, 3), "unit": "us/token/layer", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": lps * args.steps,
