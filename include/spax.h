@@ -190,6 +190,25 @@ spax_status spax_tiered_gemv(const spax_packed* h_W, const float* d_x, const int
                              int32_t* d_status, void* d_ws, size_t ws_bytes, void* stream);
 
 /*
+ * spax_masked_gemv — spax_build_mask and spax_tiered_gemv for one token in a single launch.
+ * Source: SpAx Abstract (three tiers by activation magnitude); TopK-Guided §1 and §2.1 (the
+ * threshold, TopK and guided rules); eigenradar commentary (bytes moved per token).
+ * Every CTA of the GEMV computes the token's tiers and ordered lists itself (the same rule, same
+ * results as spax_build_mask) and reads its split's columns from its own copy, so the lists never
+ * make a round trip through global memory and no second launch is needed.
+ * h_W, d_x, d_y, d_status, d_ws, ws_bytes: as spax_tiered_gemv (same workspace size and rules).
+ * h_params: host pointer, as spax_build_mask. d_tier, d_full_idx, d_approx_idx, d_counts: the
+ * mask's outputs, written exactly as spax_build_mask writes them; each may be NULL (not written).
+ * A NaN/Inf in x sets *d_status = SPAX_ERR_NONFINITE, the tiers and counts to 0 and y to 0.
+ * Requires d_in <= SPAX_MASK_MAX_DIN and the shared memory of the shape's plan to fit one CTA
+ * (else SPAX_ERR_SHAPE; every d_in up to 28672 fits).
+ */
+spax_status spax_masked_gemv(const spax_packed* h_W, const float* d_x,
+                             const spax_mask_params* h_params, float* d_y, uint8_t* d_tier,
+                             int32_t* d_full_idx, int32_t* d_approx_idx, int32_t* d_counts,
+                             int32_t* d_status, void* d_ws, size_t ws_bytes, void* stream);
+
+/*
  * spax_dense_gemv — the same-GPU dense baseline: y = W x over every column, read from the
  * bf16 full pool (W^T [d_in][d_out]) with the same kernel family as spax_tiered_gemv.
  * Source: eigenradar commentary (comparisons use dense decoding in the same weight format).

@@ -42,6 +42,9 @@ cudaError_t ensure_smem_limit(const void* kernel, int bytes) {
   return cudaSuccess;
 }
 
+// Dynamic shared memory a masked GEMV may use (227 KB per CTA, less room for static variables).
+constexpr size_t kMaskedGemvMaxSmem = 227 * 1024 - 1024;
+
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 static spax_status launch_status(cudaError_t e) {
@@ -118,12 +121,8 @@ spax_status spax_calibrate_thresholds(const float* calib_x, int n_tok, int d_in,
                                         status, ws, static_cast<cudaStream_t>(stream)));
 }
 
-spax_status spax_build_mask(const float* x, int d_in, const spax_mask_params* p, uint8_t* tier,
-                            int32_t* full_idx, int32_t* approx_idx, int32_t* counts,
-                            int32_t* status, void* stream) {
-  if (!x || !p || !tier || !full_idx || !approx_idx || !counts) return SPAX_ERR_ARG;
-  if (d_in < 1 || d_in > SPAX_MASK_MAX_DIN) return SPAX_ERR_SHAPE;
-  const spax_mask_params q = *p;
+// The rule's parameters for d_in columns (shared by the mask and the masked GEMV).
+static spax_status check_mask_params(const spax_mask_params& q, int d_in) {
   if (q.mode == SPAX_MASK_TOPK) {
     if (q.k_full < 0 || q.k_approx < 0 || (long long)q.k_full + q.k_approx > d_in)
       return SPAX_ERR_ARG;
@@ -137,6 +136,17 @@ spax_status spax_build_mask(const float* x, int d_in, const spax_mask_params* p,
   } else {
     return SPAX_ERR_ARG;
   }
+  return SPAX_OK;
+}
+
+spax_status spax_build_mask(const float* x, int d_in, const spax_mask_params* p, uint8_t* tier,
+                            int32_t* full_idx, int32_t* approx_idx, int32_t* counts,
+                            int32_t* status, void* stream) {
+  if (!x || !p || !tier || !full_idx || !approx_idx || !counts) return SPAX_ERR_ARG;
+  if (d_in < 1 || d_in > SPAX_MASK_MAX_DIN) return SPAX_ERR_SHAPE;
+  const spax_mask_params q = *p;
+  const spax_status st = check_mask_params(q, d_in);
+  if (st != SPAX_OK) return st;
   return launch_status(launch_mask(x, d_in, q, tier, full_idx, approx_idx, counts, status,
                                    static_cast<cudaStream_t>(stream)));
 }
@@ -202,6 +212,43 @@ spax_status spax_tiered_gemv(const spax_packed* W, const float* x, const int32_t
   if (!W) return SPAX_ERR_ARG;
   return gemv_common(W->d_full, W->d_approx, W->full_fmt, x, full_idx, approx_idx, counts, y,
                      W->d_out, W->d_in, status, ws, ws_bytes, stream, false);
+}
+
+spax_status spax_masked_gemv(const spax_packed* W, const float* x, const spax_mask_params* p,
+                             float* y, uint8_t* tier, int32_t* full_idx, int32_t* approx_idx,
+                             int32_t* counts, int32_t* status, void* ws, size_t ws_bytes,
+                             void* stream) {
+  if (!W || !W->d_full || !W->d_approx || !x || !p || !y) return SPAX_ERR_ARG;
+  if (W->full_fmt != SPAX_FULL_BF16 && W->full_fmt != SPAX_FULL_INT4_G128) return SPAX_ERR_ARG;
+  if (W->d_out < 128 || W->d_out % 128 != 0 || W->d_in < 1) return SPAX_ERR_SHAPE;
+  if (W->d_in > SPAX_MASK_MAX_DIN) return SPAX_ERR_SHAPE;
+  if (!aligned16(W->d_full) || !aligned16(W->d_approx) || !aligned16(y)) return SPAX_ERR_ARG;
+  const spax_mask_params q = *p;
+  const spax_status st = check_mask_params(q, W->d_in);
+  if (st != SPAX_OK) return st;
+  const int sms = sm_count_current_device();
+  if (sms < 1) return SPAX_ERR_CUDA;
+  GemvPlan pl;
+  if (!make_gemv_plan(W->d_out, W->d_in, W->full_fmt, sms, &pl)) return SPAX_ERR_SHAPE;
+  if (masked_gemv_smem_bytes(pl, W->d_in) > kMaskedGemvMaxSmem) return SPAX_ERR_SHAPE;
+  if (!ws || ws_bytes < pl.ws_bytes) return SPAX_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return SPAX_ERR_ARG;
+  GemvLaunch a;
+  a.full = W->d_full;
+  a.approx = W->d_approx;
+  a.x = x;
+  a.full_idx = nullptr;
+  a.approx_idx = nullptr;
+  a.counts = nullptr;
+  a.y = y;
+  a.status = status;
+  a.ws = ws;
+  a.d_out = W->d_out;
+  a.d_in = W->d_in;
+  a.full_fmt = W->full_fmt;
+  a.dense = false;
+  return launch_status(launch_masked_gemv(a, q, tier, full_idx, approx_idx, counts, pl,
+                                          static_cast<cudaStream_t>(stream)));
 }
 
 spax_status spax_dense_gemv(const void* Wt, const float* x, float* y, int d_out, int d_in,

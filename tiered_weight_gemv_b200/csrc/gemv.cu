@@ -30,6 +30,7 @@
 //     another) sums the S partials in split order, so results are bit-reproducible.
 #include "common.cuh"
 #include "internal.h"
+#include "select.cuh"
 
 namespace spax {
 
@@ -73,6 +74,13 @@ struct GemvParams {
   long long full_col_stride;    // bytes between full-pool columns
   long long approx_col_stride;  // bytes between approx-pool columns
   int d_out, d_in, S, G, NG;
+  // fused mask (masked GEMV only): the rule, the optional outputs, the staged-list bytes
+  spax_mask_params prm;
+  uint8_t* tier_out;
+  int32_t* fidx_out;
+  int32_t* aidx_out;
+  int32_t* counts_out;
+  int list_bytes;  // 0 for the list-driven kernels
 };
 
 // Code -> float: (word & (mask << p)) | bits(C) is the float C + code, exactly, when C = 2^(23-p)
@@ -142,15 +150,25 @@ __device__ void reduce_rows(const float* src, int cnt, int d_out, int r0, int ro
   }
 }
 
-template <int RG, int FMT, bool DENSE>
+// Shared memory of the fused kernel ahead of the GEMV's own areas: the selection's scratch and
+// keys share space with the combine and staging areas (they are dead before the GEMV starts).
+__host__ __device__ inline size_t fused_select_bytes(int d) {
+  return (sizeof(SelectSmem) + 15) / 16 * 16 + select_keys_bytes(d);
+}
+
+// FUSED: the kernel first runs the tier rule on x itself (select.cuh: every CTA computes the
+// same lists, staged in its shared memory), then reads its split's positions from there.
+template <int RG, int FMT, bool DENSE, bool FUSED>
 __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const GemvParams p) {
   using C = GemvCfg<RG>;
   constexpr int R = C::R, CG = C::CG, U = kGemvU;
   static_assert(FMT == SPAX_FULL_BF16 || !DENSE, "the dense GEMV reads the bf16 pool");
+  static_assert(!(DENSE && FUSED), "the dense GEMV has no mask");
   extern __shared__ __align__(128) uint8_t smem[];
   int32_t* meta_col_a = reinterpret_cast<int32_t*>(smem);
   int32_t* meta_col_f = meta_col_a + kGemvMeta;
-  float* red = reinterpret_cast<float*>(meta_col_f + kGemvMeta);  // [CG][kSlotFloats]
+  uint16_t* list = reinterpret_cast<uint16_t*>(meta_col_f + kGemvMeta);  // FUSED: staged lists
+  float* red = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(list) + p.list_bytes);
   __shared__ int s_bad, s_last;
 
   const int tid = threadIdx.x;
@@ -172,12 +190,63 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
     s_bad = 0;
     s_last = 0;
   }
-  pdl_wait();
-  pdl_launch_dependents();
+  int Kf, Ka;
+  uint32_t a0 = 0;  // FUSED: start of the approximate list in list[]
+  if constexpr (FUSED) {
+    // ---- the tier rule of this token, computed by every CTA (identical results) ----
+    SelectSmem& sel = *reinterpret_cast<SelectSmem*>(red);
+    uint32_t* keys = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(red) +
+                                                 (sizeof(SelectSmem) + 15) / 16 * 16);
+    select_zero(sel);
+    pdl_wait();
+    pdl_launch_dependents();
+    select_fetch(p.x, p.d_in, keys);
+    const uint32_t ts = __float_as_uint(p.prm.t_skip) & 0x7FFFFFFFu;
+    const uint32_t tf = __float_as_uint(p.prm.t_full) & 0x7FFFFFFFu;
+    uint32_t n1, n2;
+    bool bad;
+    select_pass1(p.prm.mode, p.d_in, ts, tf, keys, sel, &n1, &n2, &bad);
+    const bool lead = tile == 0 && split == 0;
+    if (bad) {  // non-finite x: every tier 0, empty lists, y = 0
+      Kf = 0;
+      Ka = 0;
+      if (lead) {
+        if (p.tier_out)
+          for (int j = tid; j < p.d_in; j += kGemvThreads) p.tier_out[j] = 0;
+        if (tid == 0) {
+          if (p.counts_out) p.counts_out[0] = p.counts_out[1] = p.counts_out[2] = p.counts_out[3] = 0;
+          record_status(p.status, SPAX_ERR_NONFINITE);
+        }
+      }
+    } else {
+      Boundary B[2];
+      select_boundaries(p.prm, p.d_in, keys, n1, n2, sel, B);
+      uint32_t nfu, nau;
+      select_compact(keys, p.d_in, B, sel, lead ? p.tier_out : nullptr, list, &nfu, &nau, &a0);
+      Kf = (int)nfu;
+      Ka = (int)nau;
+      if (tile == 0) {  // the tile-0 CTAs write the lists, each its own positions
+        const int step = S * kGemvThreads;
+        if (p.fidx_out)
+          for (int q = split + S * tid; q < Kf; q += step) p.fidx_out[q] = list[q];
+        if (p.aidx_out)
+          for (int q = split + S * tid; q < Ka; q += step) p.aidx_out[q] = list[a0 + q];
+        if (lead && tid == 0 && p.counts_out) {
+          p.counts_out[0] = Kf;
+          p.counts_out[1] = Ka;
+          p.counts_out[2] = p.prm.mode == SPAX_MASK_TOPK ? 0 : (int32_t)n1;
+          p.counts_out[3] = p.prm.mode == SPAX_MASK_TOPK ? 0 : (int32_t)n2;
+        }
+      }
+    }
+  } else {
+    pdl_wait();
+    pdl_launch_dependents();
+  }
 
   // ---- counts and (speculatively) this split's first kGemvMeta positions of both lists ----
-  int Kf, Ka;
-  if (DENSE) {
+  if constexpr (FUSED) {
+  } else if (DENSE) {
     Kf = p.d_in;
     Ka = 0;
   } else {
@@ -277,7 +346,14 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
     const int ib0 = ch * kGemvMeta;
     const int nac = max(0, min(na - ib0, kGemvMeta));
     const int nfc = max(0, min(nf - ib0, kGemvMeta));
-    if (ch > 0) {
+    if (FUSED) {
+      if (ch > 0) __syncthreads();  // every warp is done with the previous chunk's metadata
+      for (int i = tid; i < kGemvMeta; i += kGemvThreads) {
+        const int pos = split + S * (ib0 + i);
+        if (i < nac) meta_col_a[i] = list[a0 + pos];
+        if (i < nfc) meta_col_f[i] = list[pos];
+      }
+    } else if (ch > 0) {
       __syncthreads();  // every warp is done with the previous chunk's metadata
       if (!DENSE) {
         for (int i = tid; i < kGemvMeta; i += kGemvThreads) {
@@ -557,24 +633,37 @@ bool make_gemv_plan(int d_out, int d_in, int full_fmt, int sm_count, GemvPlan* p
   return true;
 }
 
-template <int RG, int FMT, bool DENSE>
-static cudaError_t launch_one(const GemvParams& gp, const GemvPlan& pl, cudaStream_t stream) {
-  using C = GemvCfg<RG>;
-  auto kern = tiered_gemv_kernel<RG, FMT, DENSE>;
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), (int)C::kSmemBytes);
+template <int RG, int FMT, bool DENSE, bool FUSED>
+static cudaError_t launch_one(const GemvParams& gp, const GemvPlan& pl, size_t smem,
+                              cudaStream_t stream) {
+  auto kern = tiered_gemv_kernel<RG, FMT, DENSE, FUSED>;
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, dim3(pl.T, pl.S), dim3(kGemvThreads), C::kSmemBytes, stream, gp);
+  return launch_pdl(kern, dim3(pl.T, pl.S), dim3(kGemvThreads), smem, stream, gp);
 }
 
-template <int FMT, bool DENSE>
-static cudaError_t launch_r(const GemvParams& gp, const GemvPlan& pl, cudaStream_t stream) {
-  if (pl.R == 512) return launch_one<1, FMT, DENSE>(gp, pl, stream);
-  if (pl.R == 1024) return launch_one<2, FMT, DENSE>(gp, pl, stream);
-  return launch_one<4, FMT, DENSE>(gp, pl, stream);
+template <int FMT, bool DENSE, bool FUSED>
+static cudaError_t launch_r(const GemvParams& gp, const GemvPlan& pl, size_t smem,
+                            cudaStream_t stream) {
+  if (pl.R == 512) return launch_one<1, FMT, DENSE, FUSED>(gp, pl, smem, stream);
+  if (pl.R == 1024) return launch_one<2, FMT, DENSE, FUSED>(gp, pl, smem, stream);
+  return launch_one<4, FMT, DENSE, FUSED>(gp, pl, smem, stream);
 }
 
-cudaError_t launch_gemv(const GemvLaunch& a, const GemvPlan& pl, cudaStream_t stream) {
-  GemvParams gp;
+static size_t gemv_smem_bytes(int R) {
+  return R == 512 ? GemvCfg<1>::kSmemBytes
+                  : (R == 1024 ? GemvCfg<2>::kSmemBytes : GemvCfg<4>::kSmemBytes);
+}
+
+size_t masked_gemv_smem_bytes(const GemvPlan& pl, int d_in) {
+  const size_t meta = size_t(2) * kGemvMeta * 4;
+  const size_t gemv = gemv_smem_bytes(pl.R) - meta;  // combine + staging areas
+  const size_t sel = fused_select_bytes(d_in);
+  return meta + select_list_bytes(d_in) + (gemv > sel ? gemv : sel);
+}
+
+static GemvParams make_params(const GemvLaunch& a, const GemvPlan& pl) {
+  GemvParams gp = {};
   uint8_t* ws = static_cast<uint8_t*>(a.ws);
   gp.full = static_cast<const uint8_t*>(a.full);
   gp.approx = static_cast<const uint8_t*>(a.approx);
@@ -596,9 +685,31 @@ cudaError_t launch_gemv(const GemvLaunch& a, const GemvPlan& pl, cudaStream_t st
   gp.S = pl.S;
   gp.G = pl.G;
   gp.NG = pl.NG;
-  if (a.dense) return launch_r<SPAX_FULL_BF16, true>(gp, pl, stream);
-  if (a.full_fmt == SPAX_FULL_BF16) return launch_r<SPAX_FULL_BF16, false>(gp, pl, stream);
-  return launch_r<SPAX_FULL_INT4_G128, false>(gp, pl, stream);
+  gp.list_bytes = 0;
+  return gp;
+}
+
+cudaError_t launch_gemv(const GemvLaunch& a, const GemvPlan& pl, cudaStream_t stream) {
+  const GemvParams gp = make_params(a, pl);
+  const size_t smem = gemv_smem_bytes(pl.R);
+  if (a.dense) return launch_r<SPAX_FULL_BF16, true, false>(gp, pl, smem, stream);
+  if (a.full_fmt == SPAX_FULL_BF16) return launch_r<SPAX_FULL_BF16, false, false>(gp, pl, smem, stream);
+  return launch_r<SPAX_FULL_INT4_G128, false, false>(gp, pl, smem, stream);
+}
+
+cudaError_t launch_masked_gemv(const GemvLaunch& a, const spax_mask_params& prm, uint8_t* tier,
+                               int32_t* full_idx, int32_t* approx_idx, int32_t* counts,
+                               const GemvPlan& pl, cudaStream_t stream) {
+  GemvParams gp = make_params(a, pl);
+  gp.prm = prm;
+  gp.tier_out = tier;
+  gp.fidx_out = full_idx;
+  gp.aidx_out = approx_idx;
+  gp.counts_out = counts;
+  gp.list_bytes = (int)select_list_bytes(a.d_in);
+  const size_t smem = masked_gemv_smem_bytes(pl, a.d_in);
+  if (a.full_fmt == SPAX_FULL_BF16) return launch_r<SPAX_FULL_BF16, false, true>(gp, pl, smem, stream);
+  return launch_r<SPAX_FULL_INT4_G128, false, true>(gp, pl, smem, stream);
 }
 
 }  // namespace spax

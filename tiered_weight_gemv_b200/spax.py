@@ -58,6 +58,8 @@ _SIGS = {
     "spax_build_mask": ([_P, _I, ctypes.POINTER(spax_mask_params), _P, _P, _P, _P, _P, _P], _I),
     "spax_tiered_gemv": ([ctypes.POINTER(spax_packed), _P, _P, _P, _P, _P, _P, _P, _Z, _P], _I),
     "spax_dense_gemv": ([_P, _P, _P, _I, _I, _P, _P, _Z, _P], _I),
+    "spax_masked_gemv": ([ctypes.POINTER(spax_packed), _P, ctypes.POINTER(spax_mask_params), _P,
+                          _P, _P, _P, _P, _P, _P, _Z, _P], _I),
     "spax_tiered_gemv_fixed_scratch": ([ctypes.POINTER(spax_packed), _P, _P, _P, _P, _P, _P, _P],
                                        _I),
     "spax_fixed_scratch_bytes": ([], _Z),
@@ -214,6 +216,24 @@ def spax_tiered_gemv(W: PackedMatrix, x: torch.Tensor, full_idx: torch.Tensor,
         _dev(approx_idx, torch.int32, "approx_idx"), _dev(counts, torch.int32, "counts"),
         _dev(y, torch.float32, "y"), _dev(status, torch.int32, "status"), _dev(ws, None, "ws"),
         ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def spax_masked_gemv(W: PackedMatrix, x: torch.Tensor, params: spax_mask_params, y: torch.Tensor,
+                     status: torch.Tensor, ws: torch.Tensor, tier=None, full_idx=None,
+                     approx_idx=None, counts=None, stream=None, desc=None) -> None:
+    """The mask and the tiered GEMV in one launch; tier / lists / counts are optional outputs."""
+    if x.numel() != W.d_in or y.numel() != W.d_out:
+        raise ValueError("x / y sizes do not match W")
+    for t, n in ((tier, W.d_in), (full_idx, W.d_in), (approx_idx, W.d_in), (counts, 4)):
+        if t is not None and t.numel() < n:
+            raise ValueError("mask output too small")
+    d = W.desc() if desc is None else desc
+    _check("spax_masked_gemv", _lib.spax_masked_gemv(
+        ctypes.byref(d), _dev(x, torch.float32, "x"), ctypes.byref(params),
+        _dev(y, torch.float32, "y"), _dev(tier, torch.uint8, "tier"),
+        _dev(full_idx, torch.int32, "full_idx"), _dev(approx_idx, torch.int32, "approx_idx"),
+        _dev(counts, torch.int32, "counts"), _dev(status, torch.int32, "status"),
+        _dev(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def spax_tiered_gemv_fixed_scratch(W: PackedMatrix, x: torch.Tensor, full_idx: torch.Tensor,
