@@ -103,27 +103,29 @@ __device__ __forceinline__ uint32_t ld_stream16(const uint8_t* p) {
 }
 
 // Fixed-order sum of `cnt` partial rows [r0, r0+rows) (row stride d_out), written to dst + r0.
-// The partials are cut into consecutive batches of kBatch, each summed by one thread with all
-// its loads in flight; the batch sums are then added in batch order. The association depends only
-// on cnt, so the result is reproducible.
+// The partials are cut into consecutive batches of kb, sized so that every thread of the CTA has
+// one item (a float4 of one batch) with all its loads in flight; the batch sums are then added in
+// batch order. The association depends only on cnt and rows, so the result is reproducible.
 template <int NT>
 __device__ void reduce_rows(const float* src, int cnt, int d_out, int r0, int rows, float* dst,
-                            int tid, float4* scratch /* [nbatch][rows/4] */) {
-  constexpr int kBatch = 16;
+                            int tid, float4* scratch /* [nb][rows/4] */) {
+  constexpr int kMaxBatch = 16;
   const int n4 = rows >> 2;
-  const int nb = (cnt + kBatch - 1) / kBatch;  // <= 3 when cnt <= 48
+  int nb = max(1, NT / max(n4, 1));
+  const int kb = min(kMaxBatch, (cnt + nb - 1) / nb);
+  nb = (cnt + kb - 1) / kb;
   const size_t stride4 = static_cast<size_t>(d_out) >> 2;
   const float4* s4 = reinterpret_cast<const float4*>(src + r0);
   for (int item = tid; item < n4 * nb; item += NT) {
     const int i = item % n4, b = item / n4;
-    const int k0 = b * kBatch, kn = min(cnt - k0, kBatch);
-    float4 v[kBatch];
+    const int k0 = b * kb, kn = min(cnt - k0, kb);
+    float4 v[kMaxBatch];
 #pragma unroll
-    for (int k = 0; k < kBatch; ++k)
+    for (int k = 0; k < kMaxBatch; ++k)
       if (k < kn) v[k] = __ldcg(s4 + (size_t)(k0 + k) * stride4 + i);
     float4 acc = v[0];
 #pragma unroll
-    for (int k = 1; k < kBatch; ++k)
+    for (int k = 1; k < kMaxBatch; ++k)
       if (k < kn) {
         acc.x += v[k].x;
         acc.y += v[k].y;
@@ -148,6 +150,19 @@ __device__ void reduce_rows(const float* src, int cnt, int d_out, int r0, int ro
     }
     reinterpret_cast<float4*>(dst + r0)[i] = acc;
   }
+}
+
+// Arrival ticket of a split-K group: after a CTA barrier (every thread's partial stores are done),
+// one thread adds 1 with acquire-release semantics at GPU scope. The release publishes the whole
+// CTA's stores (they happen before it through the barrier); the last arrival's acquire makes every
+// other CTA's partials visible to it (and, through the next barrier, to its threads). The last
+// arrival resets the counter for the next call.
+__device__ __forceinline__ bool ticket_last(uint32_t* t, uint32_t n) {
+  uint32_t old;
+  asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(old) : "l"(t) : "memory");
+  const bool last = old == n - 1;
+  if (last) *t = 0u;
+  return last;
 }
 
 // Shared memory of the fused kernel ahead of the GEMV's own areas: the selection's scratch and
@@ -557,35 +572,19 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
   const int grp = split / p.G;
   const int gbeg = grp * p.G;
   const int gsz = min(p.G, S - gbeg);
-  float4* scratch = reinterpret_cast<float4*>(red);  // [<=4][R/4] fits in CG >= 4 slots
-  __threadfence();
+  float4* scratch = reinterpret_cast<float4*>(red);  // [nb][R/4]: at most 24 KB, fits the slots
   __syncthreads();
-  if (tid == 0) {
-    uint32_t* t = p.gtick + (size_t)tile * p.NG + grp;
-    const uint32_t old = atomicAdd(t, 1u);
-    const int last = (old == (uint32_t)(gsz - 1));
-    if (last) *t = 0u;  // every other split of the group has arrived: reset for the next call
-    s_last = last;
-  }
+  if (tid == 0) s_last = ticket_last(p.gtick + (size_t)tile * p.NG + grp, (uint32_t)gsz);
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   float* gdst = (p.NG == 1) ? p.y : p.gpart + (size_t)grp * p.d_out;
   reduce_rows<kGemvThreads>(p.part + (size_t)gbeg * p.d_out, gsz, p.d_out, r0, rows_here, gdst,
                             tid, scratch);
   if (p.NG == 1) return;
-  __threadfence();
   __syncthreads();
-  if (tid == 0) {
-    uint32_t* t = p.ttick + tile;
-    const uint32_t old = atomicAdd(t, 1u);
-    const int last = (old == (uint32_t)(p.NG - 1));
-    if (last) *t = 0u;
-    s_last = last;
-  }
+  if (tid == 0) s_last = ticket_last(p.ttick + tile, (uint32_t)p.NG);
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   reduce_rows<kGemvThreads>(p.gpart, p.NG, p.d_out, r0, rows_here, p.y, tid, scratch);
 }
 

@@ -52,8 +52,8 @@ struct SelectSmem {
   uint32_t hb[2][512];   // bits 8..0 under a 22-bit prefix (when pass 2 leaves V open)
   uint32_t stat[4];      // #keys < t_skip, #keys < t_full, non-finite flag
   uint32_t sel[2][4];    // per boundary: prefix / key, count above, count in the bin
-  uint32_t wsum[kSelWarps];
-  uint32_t wscan[kSelWarps];
+  alignas(16) uint32_t wsum[kSelWarps];
+  alignas(16) uint32_t wscan[kSelWarps];
   uint32_t flag[2];
 };
 
@@ -215,7 +215,14 @@ __device__ __forceinline__ void block_find_pair(const uint32_t* h0, const uint32
   if (lane == 31) S.wsum[wid] = incl;
   __syncthreads();
   uint32_t cum = (t ? ab1 : ab0) + incl - s;
-  for (int w = 8 * t; w < wid; ++w) cum += S.wsum[w];
+  {  // counts of the warps before this one in its half (8 per half), as two vector loads
+    const uint4 lo = *reinterpret_cast<const uint4*>(&S.wsum[8 * t]);
+    const uint4 hi = *reinterpret_cast<const uint4*>(&S.wsum[8 * t + 4]);
+    const uint32_t w8[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+    const int wl = wid - 8 * t;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) cum += w < wl ? w8[w] : 0u;
+  }
   const uint32_t K = t ? K1 : K0;
   if ((t ? act1 : act0) && cum < K && K <= cum + s) {
     uint32_t a = cum;
@@ -280,7 +287,12 @@ __device__ __forceinline__ void select_boundaries(const spax_mask_params& prm, i
       if (lane == 31) S.wsum[wid] = incl;
       __syncthreads();
       uint32_t cum = incl - s;
-      for (int w = 0; w < wid; ++w) cum += S.wsum[w];
+#pragma unroll
+      for (int g = 0; g < kSelWarps / 4; ++g) {  // counts of the warps before this one
+        const uint4 q = *reinterpret_cast<const uint4*>(&S.wsum[4 * g]);
+        cum += (4 * g + 0 < wid ? q.x : 0u) + (4 * g + 1 < wid ? q.y : 0u) +
+               (4 * g + 2 < wid ? q.z : 0u) + (4 * g + 3 < wid ? q.w : 0u);
+      }
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
         const uint32_t K = t ? K1 : K0;
