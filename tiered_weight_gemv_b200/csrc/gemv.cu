@@ -233,6 +233,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
           record_status(p.status, SPAX_ERR_NONFINITE);
         }
       }
+      __syncthreads();  // the selection's scratch is dead before the combine area reuses it
     } else {
       Boundary B[2];
       select_boundaries(p.prm, p.d_in, keys, n1, n2, sel, B);
@@ -282,7 +283,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
   }
   const int nf = Kf > split ? (Kf - split + S - 1) / S : 0;  // items of this split
   const int na = Ka > split ? (Ka - split + S - 1) / S : 0;
-  const int nchunks = (max(nf, na) + kGemvMeta - 1) / kGemvMeta;
+  const int nchunks = FUSED ? ((nf | na) ? 1 : 0) : (max(nf, na) + kGemvMeta - 1) / kGemvMeta;
 
   // this warp's slice of the packed pools
   const long long off_full = 2LL * (rb + 8 * lane);  // bf16 pool
@@ -298,7 +299,18 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
   // 2-bit Σ x*scale and Σ x*min, int4 Σ x*scale (reduced over the warp at the end)
   float sA[4] = {0.f, 0.f, 0.f, 0.f}, bA[4] = {0.f, 0.f, 0.f, 0.f}, s4[4] = {0.f, 0.f, 0.f, 0.f};
 
-  // Stage nb (<= kBatch2) 2-bit records of columns meta_col_a[cg + CG*(k0 + k)] and prepare
+  // Column of local position i of this split's approximate / full list (in the current chunk):
+  // the fused kernel reads its staged lists directly, the list-driven one its metadata arrays.
+  auto colA = [&](int i) -> int {
+    if constexpr (FUSED) return (int)list[a0 + split + S * i];
+    else return meta_col_a[i];
+  };
+  auto colF = [&](int i) -> int {
+    if constexpr (FUSED) return (int)list[split + S * i];
+    else return meta_col_f[i];
+  };
+
+  // Stage nb (<= kBatch2) 2-bit records of columns colA(cg + CG*(k0 + k)) and prepare
   // their coefficients c[k][g] = x*scale_g (lane k), accumulating the group sums.
   auto stage_approx = [&](int k0, int nb) {
     __syncwarp();
@@ -307,13 +319,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
 #pragma unroll
     for (int t = 0; t < kChunks2; ++t) {
       const int q = t * 32 + lane, k = q / 9, piece = q - 9 * k;
-      const int col = k < nb ? max(meta_col_a[cg + CG * (k0 + k)], 0) : 0;
+      const int col = k < nb ? max(colA(cg + CG * (k0 + k)), 0) : 0;
       v[t] = k < nb ? ld_stream128(p.approx + col * p.approx_col_stride + off_approx + 16 * piece)
                     : make_uint4(0u, 0u, 0u, 0u);
     }
     float xk = 0.f;
     if (lane < nb) {
-      const int col = meta_col_a[cg + CG * (k0 + lane)];
+      const int col = colA(cg + CG * (k0 + lane));
       xk = col >= 0 ? __ldg(p.x + col) : 0.f;  // an invalid column contributes zero
     }
 #pragma unroll
@@ -359,16 +371,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
 
   for (int ch = 0; ch < nchunks; ++ch) {
     const int ib0 = ch * kGemvMeta;
-    const int nac = max(0, min(na - ib0, kGemvMeta));
-    const int nfc = max(0, min(nf - ib0, kGemvMeta));
-    if (FUSED) {
-      if (ch > 0) __syncthreads();  // every warp is done with the previous chunk's metadata
-      for (int i = tid; i < kGemvMeta; i += kGemvThreads) {
-        const int pos = split + S * (ib0 + i);
-        if (i < nac) meta_col_a[i] = list[a0 + pos];
-        if (i < nfc) meta_col_f[i] = list[pos];
-      }
-    } else if (ch > 0) {
+    const int nac = FUSED ? na : max(0, min(na - ib0, kGemvMeta));
+    const int nfc = FUSED ? nf : max(0, min(nf - ib0, kGemvMeta));
+    if constexpr (!FUSED) {
+    if (ch > 0) {
       __syncthreads();  // every warp is done with the previous chunk's metadata
       if (!DENSE) {
         for (int i = tid; i < kGemvMeta; i += kGemvThreads) {
@@ -378,7 +384,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
         }
       }
     }
-    // validate this chunk's columns (the dense GEMV generates them); an invalid one becomes -1
+    // validate this chunk's columns (the dense GEMV generates them); an invalid one becomes -1.
+    // (The fused kernel's lists come from its own selection: nothing to copy or check.)
     for (int i = tid; i < kGemvMeta; i += kGemvThreads) {
       if (i < nac && (unsigned)meta_col_a[i] >= (unsigned)p.d_in) {
         s_bad = 1;
@@ -392,6 +399,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
       }
     }
     __syncthreads();
+    }
     if (!wrows) continue;
     const int nAw = nac > cg ? (nac - cg + CG - 1) / CG : 0;  // this warp's 2-bit columns
     const int nFw = nfc > cg ? (nfc - cg + CG - 1) / CG : 0;  // this warp's full columns
@@ -407,7 +415,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
         float xf[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-          int col = u < nfb ? meta_col_f[cg + CG * (kf + u)] : -1;
+          int col = u < nfb ? colF(cg + CG * (kf + u)) : -1;
           xf[u] = col >= 0 ? __ldg(p.x + col) : 0.f;
           const uint8_t* src = p.full + max(col, 0) * p.full_col_stride + off_full;
           w0[u] = (u < nfb && v0) ? ld_stream128(src) : make_uint4(0u, 0u, 0u, 0u);
@@ -458,7 +466,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
 #pragma unroll
         for (int t = 0; t < 9; ++t) {
           const int q = t * 32 + lane, k = q / 17, piece = q - 17 * k;
-          const int col = k < nb ? max(meta_col_f[cg + CG * (kf + k)], 0) : 0;
+          const int col = k < nb ? max(colF(cg + CG * (kf + k)), 0) : 0;
           const uint8_t* src = p.full + col * p.full_col_stride;
           v[t] = (q < 17 * kBatch4 && k < nb)
                      ? ld_stream128(piece < 16 ? src + nib0 + 16 * piece : src + scl0)
@@ -466,7 +474,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
         }
         float xk = 0.f;
         if (lane < nb) {
-          const int col = meta_col_f[cg + CG * (kf + lane)];
+          const int col = colF(cg + CG * (kf + lane));
           xk = col >= 0 ? __ldg(p.x + col) : 0.f;
         }
 #pragma unroll
