@@ -269,6 +269,31 @@ spax_status spax_block_budgets(const double* h_sens, int n_blocks, double s, dou
                                double lo, double hi, double* h_s_out);
 
 /*
+ * Block output reconstruction error for the per-matrix sparsities h_p[0, n) of one block
+ * (measured by the caller, e.g. on calibration tokens); ctx is passed through unchanged.
+ */
+typedef double (*spax_block_error_fn)(const double* h_p, int n, void* ctx);
+
+/*
+ * spax_greedy_allocation — host-only: per-matrix sparsities inside one block, given the block's
+ * budget (TopK-Guided, Appendix D "Block-wise Greedy Sparsity Allocation", and Table 4).
+ * Matrix m has parameter count h_params[m] = f_m and step alpha_m = alpha * fbar / f_m (fbar
+ * the mean count), so one increment of any matrix moves the compute-weighted block sparsity
+ * P = sum_m f_m p_m / sum_m f_m by alpha / n. From p = 0, each step tries the next increment of
+ * every matrix whose p_m + alpha_m stays <= p_max, evaluates err on each candidate allocation,
+ * and keeps the candidate with the least error (ties: the lower matrix index). It stops as soon
+ * as P >= p_target - 1e-12. Writes h_p_out[n], *h_steps and, when h_order is not NULL, the
+ * matrix chosen at each step (h_order holds max_steps entries).
+ * Requires n >= 1, every f_m > 0, alpha > 0, 0 <= p_target <= p_max <= 1 and err != NULL.
+ * Returns SPAX_ERR_ARG if the budget cannot be reached within max_steps steps or before every
+ * matrix is at p_max (the allocation reached so far is still written).
+ */
+spax_status spax_greedy_allocation(const double* h_params, int n, double alpha, double p_target,
+                                   double p_max, spax_block_error_fn err, void* ctx,
+                                   int max_steps, double* h_p_out, int32_t* h_order,
+                                   int32_t* h_steps);
+
+/*
  * Host-only byte account of one tiered GEMV (eigenradar "bytes moved per generated token"):
  * weight bytes the kernel must read for n_full full and n_approx approximate columns of a
  * d_out-row matrix: n_full * (2*d_out for bf16 | 0.5*d_out + 2*d_out/128 for int4) +

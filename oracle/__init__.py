@@ -257,6 +257,39 @@ def block_budgets(sens, s, lam, lo=0.05, hi=0.95):
     return out
 
 
+def greedy_allocation(params, alpha, p_target, err, p_max=1.0, step_base="mean", max_steps=100000):
+    """Block-wise greedy per-matrix sparsity (TopK-Guided, Appendix D and Table 4), written out
+    step by step: every matrix m has step alpha * base / f_m (base = the mean parameter count, or
+    the total for step_base="sum": the pages do not say which, and Table 4 fits both); each round
+    tries the next increment of every matrix that stays within p_max, keeps the one with the least
+    block error err(p) (first index on a tie) and stops once the compute-weighted sparsity
+    sum f_m p_m / sum f_m reaches p_target. Returns (p, order, reached)."""
+    f = [float(v) for v in params]
+    n = len(f)
+    total = sum(f)
+    base = total / n if step_base == "mean" else total
+    steps = [alpha * base / fm for fm in f]
+    p = [0.0] * n
+    order = []
+    while sum(fm * pm for fm, pm in zip(f, p)) / total < p_target - 1e-12:
+        if len(order) >= max_steps:
+            return np.array(p), order, False
+        best, best_err = -1, 0.0
+        for m in range(n):
+            if p[m] + steps[m] > p_max + 1e-12:
+                continue
+            cand = list(p)
+            cand[m] += steps[m]
+            e = float(err(np.array(cand)))
+            if best < 0 or e < best_err:
+                best, best_err = m, e
+        if best < 0:
+            return np.array(p), order, False
+        p[best] += steps[best]
+        order.append(best)
+    return np.array(p), order, True
+
+
 def weight_bytes(d_out: int, fmt: int, n_full: int, n_approx: int) -> int:
     """Bytes the tiered product reads for one token (eigenradar: bytes moved per token)."""
     return int(_L().oracle_weight_bytes(d_out, fmt, n_full, n_approx))

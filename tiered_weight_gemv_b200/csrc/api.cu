@@ -5,6 +5,7 @@
 #include <cstring>
 #include <mutex>
 #include <unordered_map>
+#include <vector>
 
 #include "common.cuh"
 #include "internal.h"
@@ -301,6 +302,55 @@ spax_status spax_block_budgets(const double* sens, int n, double s, double lambd
     out[b] = v < lo ? lo : (v > hi ? hi : v);
   }
   return SPAX_OK;
+}
+
+spax_status spax_greedy_allocation(const double* f, int n, double alpha, double p_target,
+                                   double p_max, spax_block_error_fn err, void* ctx,
+                                   int max_steps, double* p_out, int32_t* order,
+                                   int32_t* steps) {
+  if (!f || !p_out || !steps || !err || n < 1 || max_steps < 0) return SPAX_ERR_ARG;
+  if (!(alpha > 0.0) || !(p_target >= 0.0) || !(p_target <= p_max) || !(p_max <= 1.0))
+    return SPAX_ERR_ARG;
+  double fsum = 0.0;
+  for (int m = 0; m < n; ++m) {
+    if (!(f[m] > 0.0) || !std::isfinite(f[m])) return SPAX_ERR_ARG;
+    fsum += f[m];
+  }
+  const double fbar = fsum / n;
+  std::vector<double> p(n, 0.0), cand(n);
+  *steps = 0;
+  spax_status st = SPAX_OK;
+  for (;;) {
+    double P = 0.0;
+    for (int m = 0; m < n; ++m) P += f[m] * p[m];
+    if (P / fsum >= p_target - 1e-12) break;
+    if (*steps >= max_steps) {
+      st = SPAX_ERR_ARG;
+      break;
+    }
+    int best = -1;
+    double best_err = 0.0;
+    for (int m = 0; m < n; ++m) {
+      const double step = alpha * fbar / f[m];
+      if (p[m] + step > p_max + 1e-12) continue;
+      cand = p;
+      cand[m] += step;
+      const double e = err(cand.data(), n, ctx);
+      if (best < 0 || e < best_err) {
+        best = m;
+        best_err = e;
+      }
+    }
+    if (best < 0) {  // every matrix is at its ceiling
+      st = SPAX_ERR_ARG;
+      break;
+    }
+    p[best] += alpha * fbar / f[best];
+    if (order) order[*steps] = best;
+    ++*steps;
+  }
+  for (int m = 0; m < n; ++m) p_out[m] = p[m];
+  return st;
 }
 
 uint64_t spax_weight_bytes(int d_out, int full_fmt, int64_t n_full, int64_t n_approx) {

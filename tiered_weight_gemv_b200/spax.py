@@ -68,6 +68,8 @@ _SIGS = {
     "spax_block_budgets": ([_P, _I, ctypes.c_double, ctypes.c_double, ctypes.c_double,
                             ctypes.c_double, _P], _I),
     "spax_weight_bytes": ([_I, _I, ctypes.c_int64, ctypes.c_int64], ctypes.c_uint64),
+    "spax_greedy_allocation": ([_P, _I, ctypes.c_double, ctypes.c_double, ctypes.c_double, _P, _P,
+                                _I, _P, _P, _P], _I),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -134,6 +136,26 @@ def spax_block_budgets(sens, s: float, lam: float, lo: float = 0.05, hi: float =
     _check("spax_block_budgets", _lib.spax_block_budgets(
         sens.ctypes.data_as(_P), sens.size, s, lam, lo, hi, out.ctypes.data_as(_P)))
     return out
+
+
+BLOCK_ERROR_FN = ctypes.CFUNCTYPE(ctypes.c_double, ctypes.POINTER(ctypes.c_double), ctypes.c_int,
+                                  ctypes.c_void_p)
+
+
+def spax_greedy_allocation(params, alpha: float, p_target: float, err, p_max: float = 1.0,
+                           max_steps: int = 100000):
+    """Per-matrix sparsities of one block (the library's greedy allocation). err(p) -> block
+    error for a numpy array of per-matrix sparsities. Returns (p, order)."""
+    f = np.ascontiguousarray(params, dtype=np.float64)
+    n = f.size
+    cb = BLOCK_ERROR_FN(lambda pp, nn, ctx: float(err(np.ctypeslib.as_array(pp, (nn,)).copy())))
+    p = np.zeros(n, np.float64)
+    order = np.zeros(max(1, max_steps), np.int32)
+    steps = ctypes.c_int32(0)
+    _check("spax_greedy_allocation", _lib.spax_greedy_allocation(
+        f.ctypes.data_as(_P), n, alpha, p_target, p_max, ctypes.cast(cb, _P), None, max_steps,
+        p.ctypes.data_as(_P), order.ctypes.data_as(_P), ctypes.byref(steps)))
+    return p, order[: steps.value].copy()
 
 
 def spax_weight_bytes(d_out: int, full_fmt: int, n_full: int, n_approx: int) -> int:
