@@ -395,6 +395,156 @@ def run_gpu(args, rank, world, local):
     return res, sites, tot_bytes, tot_ms, launches_per_step, h2d, d2h, sampler.summary(), host
 
 
+# ----------------------------------------------------------------------------- extra measurements
+
+LLAMA3_SITES = [("qkv", 6144, 4096, 201), ("o", 4096, 4096, 202), ("gate_up", 28672, 4096, 203),
+                ("down", 4096, 14336, 204)]
+LLAMA3_POINTS = [(f, a) for f in (0.1, 0.2, 0.3) for a in (0.2, 0.3)]
+L2_BYTES = 126 * 2 ** 20
+
+
+def _replicas_for(bytes_per_replica: float) -> int:
+    """Weight replicas so that a round robin over them reads at least 3x L2 between reuses."""
+    return max(4, math.ceil(3 * L2_BYTES / bytes_per_replica))
+
+
+def run_extras(args, dev):
+    """Measurements beside the headline, on one GPU (each a CUDA graph of n tokens, timed like the
+    headline): dequantisation against loading, the Llama-3-8B (full, approx) sweep with its
+    c0 + bytes/BW fit, and the dense kernels (this library's and torch.mv / cuBLAS) on the same
+    layer."""
+    from tiered_weight_gemv_b200 import spax, synth
+
+    n_tok = 16
+    steps, warmup = max(5, min(args.steps, 20)), args.warmup
+    stream = torch.cuda.Stream(device=dev)
+    out = {}
+
+    def packed_replicas(W, d_out, d_in, n_rep):
+        pm = spax.alloc_packed(d_out, d_in, spax.FULL_BF16, device=dev)
+        spax.spax_pack_weights(W, spax.FULL_BF16, pm)
+        return [pm] + [spax.PackedMatrix(d_out, d_in, spax.FULL_BF16, pm.full.clone(),
+                                         pm.approx.clone()) for _ in range(n_rep - 1)]
+
+    def timed(fn):
+        with torch.cuda.stream(stream):
+            fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        ms = time_graph(g, steps, warmup, stream)
+        del g
+        return ms
+
+    # ---- dequantisation against loading: all bf16, all 2-bit, mixed, 2-bit from L2 ----
+    dq = {}
+    for label, d_out, d_in, tid in [("proj_4096x4096", 4096, 4096, 301),
+                                    ("gate_up_22016x4096", 22016, 4096, 302)]:
+        W = synth.weight(d_out, d_in, 6, tid, device=dev)
+        reps = packed_replicas(W, d_out, d_in, _replicas_for(2.3 * d_out * d_in))
+        del W
+        X = synth.laplace((n_tok, d_in), 6, tid + 10, device=dev)
+        y = torch.empty(n_tok, d_out, device=dev)
+        st = torch.zeros(1, dtype=torch.int32, device=dev)
+        ws = spax.alloc_workspace(spax.OP_TIERED_GEMV, d_out, d_in, device=dev)
+        descs = [pm.desc() for pm in reps]
+        q = int(math.floor(0.25 * d_in + 0.5))
+        cases = [("all_full", d_in, 0, True), ("all_approx", 0, d_in, True),
+                 ("mixed_25_25", q, q, True), ("all_approx_l2_resident", 0, d_in, False)]
+        rows = {}
+        for case, kf, ka, rotate in cases:
+            prm = spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka)
+
+            def fn(prm=prm, rotate=rotate):
+                for t in range(n_tok):
+                    r = t % len(reps) if rotate else 0
+                    spax.spax_masked_gemv(reps[r], X[t], prm, y[t], st, ws, desc=descs[r])
+
+            ms = timed(fn)
+            by = fused_bytes(d_out, d_in, kf, ka)
+            rows[case] = {"us": round(ms * 1000 / n_tok, 3), "bytes": by,
+                          "GBps": round(by * n_tok / (ms * 1e-3) / 1e9, 1)}
+        if int(st.item()) != 0:
+            raise RuntimeError(f"device status {int(st.item())} in the dequant runs ({label})")
+        rows["replicas"] = len(reps)
+        dq[label] = rows
+        del reps, descs, ws, X, y
+        torch.cuda.empty_cache()
+    out["dequant_vs_load"] = dq
+
+    # ---- Llama-3-8B layer: the six (full, approx) points, dense, torch.mv ----
+    per_rep = sum(2.3 * d_out * d_in for _, d_out, d_in, _ in LLAMA3_SITES)
+    n_rep = _replicas_for(per_rep)
+    layer = {}
+    for name, d_out, d_in, tid in LLAMA3_SITES:
+        W = synth.weight(d_out, d_in, 7, tid, device=dev)
+        reps = packed_replicas(W, d_out, d_in, n_rep)
+        del W
+        layer[name] = dict(reps=reps, descs=[pm.desc() for pm in reps],
+                           X=synth.laplace((n_tok, d_in), 7, tid + 10, device=dev),
+                           y=torch.empty(n_tok, d_out, device=dev),
+                           st=torch.zeros(1, dtype=torch.int32, device=dev),
+                           ws=spax.alloc_workspace(spax.OP_TIERED_GEMV, d_out, d_in, device=dev),
+                           dws=spax.alloc_workspace(spax.OP_DENSE_GEMV, d_out, d_in, device=dev))
+        layer[name]["Xh"] = layer[name]["X"].to(torch.bfloat16)
+    torch.cuda.synchronize()
+    points = []
+    for f, a in LLAMA3_POINTS:
+        prms = {name: spax.mask_params(spax.MASK_TOPK, k_full=int(math.floor(f * d_in + 0.5)),
+                                       k_approx=int(math.floor(a * d_in + 0.5)))
+                for name, _, d_in, _ in LLAMA3_SITES}
+
+        def fn(prms=prms):
+            for t in range(n_tok):
+                for name, *_ in LLAMA3_SITES:
+                    L = layer[name]
+                    r = t % n_rep
+                    spax.spax_masked_gemv(L["reps"][r], L["X"][t], prms[name], L["y"][t], L["st"],
+                                          L["ws"], desc=L["descs"][r])
+
+        ms = timed(fn)
+        by = sum(fused_bytes(d_out, d_in, prms[n].k_full, prms[n].k_approx)
+                 for n, d_out, d_in, _ in LLAMA3_SITES)
+        points.append({"full": f, "approx": a, "us_per_token_layer": round(ms * 1000 / n_tok, 3),
+                       "bytes_per_token_layer": by,
+                       "GBps": round(by * n_tok / (ms * 1e-3) / 1e9, 1)})
+    for name, *_ in LLAMA3_SITES:
+        if int(layer[name]["st"].item()) != 0:
+            raise RuntimeError(f"device status {int(layer[name]['st'].item())} in the sweep ({name})")
+
+    def dense_fn():
+        for t in range(n_tok):
+            for name, d_out, d_in, _ in LLAMA3_SITES:
+                L = layer[name]
+                spax.spax_dense_gemv(L["reps"][t % n_rep].full, L["X"][t], L["y"][t], d_out, d_in,
+                                     L["st"], L["dws"])
+
+    def torch_mv_fn():
+        for t in range(n_tok):
+            for name, d_out, d_in, _ in LLAMA3_SITES:
+                L = layer[name]
+                Wt = L["reps"][t % n_rep].full.view(torch.bfloat16).view(d_in, d_out)
+                torch.mv(Wt.t(), L["Xh"][t])
+
+    dense_bytes = sum(2 * d_out * d_in for _, d_out, d_in, _ in LLAMA3_SITES)
+    ms_dense = timed(dense_fn)
+    ms_mv = timed(torch_mv_fn)
+    out["llama3_8b_layer_sweep"] = {
+        "sites": {n: [d_out, d_in] for n, d_out, d_in, _ in LLAMA3_SITES},
+        "tokens": n_tok, "replicas": n_rep, "points": points,
+        "fit_time_vs_bytes": fit_c0_bw([(p["bytes_per_token_layer"], p["us_per_token_layer"])
+                                        for p in points]),
+        "dense_us_per_token_layer": round(ms_dense * 1000 / n_tok, 3),
+        "dense_GBps": round(dense_bytes * n_tok / (ms_dense * 1e-3) / 1e9, 1),
+        "torch_mv_bf16_us_per_token_layer": round(ms_mv * 1000 / n_tok, 3),
+        "torch_mv_note": "cuBLAS through torch.mv on the same bf16 pool with bf16 x (sanity figure)",
+    }
+    del layer
+    torch.cuda.empty_cache()
+    return out
+
+
 def fit_c0_bw(points):
     """Least-squares time = c0 + bytes / BW over (bytes, us) points: the fixed per-launch cost and
     the streaming rate (the byte-account method of the ByteCross abstract)."""
@@ -472,16 +622,28 @@ class OracleRunner:
             o.tiered_gemv(*self.pools[name], o.FULL_BF16, d_out, d_in, self.xs[name][t], tier)
 
 
-def cpu_baseline(n_tokens, mats, xs):
+def cpu_baseline(n_tokens, mats, xs, omp=True):
     r = OracleRunner(mats, xs)
     t0 = time.perf_counter()
     for t in range(n_tokens):
         r.token(t)
     dt = time.perf_counter() - t0
-    return {"value": round(dt * 1e6 / n_tokens, 1), "unit": "us/token/layer", "cores": 1,
-            "kind": "oracle",
-            "sample": f"{n_tokens} of the {N_TOKENS} tokens, all four sites, single-threaded C "
-                      f"oracle (fp64), {dt:.1f} s"}
+    res = {"value": round(dt * 1e6 / n_tokens, 1), "unit": "us/token/layer", "cores": 1,
+           "kind": "oracle",
+           "sample": f"{n_tokens} of the {N_TOKENS} tokens, all four sites, single-threaded C "
+                     f"oracle (fp64), {dt:.1f} s"}
+    if omp:  # the same oracle source built with OpenMP: row chunks over every host core
+        threads = r.o.use_openmp(True)
+        try:
+            t0 = time.perf_counter()
+            for t in range(n_tokens):
+                r.token(t)
+            dto = time.perf_counter() - t0
+        finally:
+            r.o.use_openmp(False)
+        res["openmp"] = {"value": round(dto * 1e6 / n_tokens, 1), "unit": "us/token/layer",
+                         "cores": threads, "sample": f"the same {n_tokens} tokens, {dto:.1f} s"}
+    return res
 
 
 def run_reference(args, rank, world):
@@ -527,6 +689,9 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=24)
     ap.add_argument("--ref-tokens", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the measurements beside the headline (dequant vs load, the "
+                         "Llama-3-8B sweep and fit, dense and torch.mv)")
     ap.add_argument("--sites", default="", help="comma-separated subset of qkv,o,gate_up,down "
                     "(profiling runs); the default runs the whole block")
     args = ap.parse_args()
@@ -578,6 +743,8 @@ def main():
             "gpu_launches": lps * args.steps,
             "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
         }
+        if world == 1 and not args.no_extras and not args.sites:
+            line["extras"] = run_extras(args, torch.device("cuda", local))
         if host is not None:
             line["cpu_baseline"] = cpu_baseline(args.cpu_tokens, *host)
         if rank == 0:

@@ -64,7 +64,8 @@ typedef enum {
   SPAX_ERR_WORKSPACE = 3,  /* workspace pointer NULL or ws_bytes too small */
   SPAX_ERR_CUDA = 4,       /* a CUDA runtime call or launch failed */
   SPAX_ERR_NONFINITE = 5,  /* device: an input activation was NaN or Inf */
-  SPAX_ERR_TIMEOUT = 6,    /* device: a bounded pipeline wait ran out (a library bug) */
+  SPAX_ERR_TIMEOUT = 6,    /* device: a bounded wait ran out (a split's partial sums never
+                              arrived: a library bug, or the grid could not be resident at once) */
   SPAX_ERR_INDEX = 7       /* device: counts or a column index out of range */
 } spax_status;
 
@@ -180,10 +181,12 @@ spax_status spax_build_mask(const float* d_x, int d_in, const spax_mask_params* 
  * counts on the device; no host sync). d_y fp32 [d_out] (device), fully written.
  * Accumulation is fp32, split over CTAs, then reduced in a fixed order (bit-reproducible for a
  * given GPU model and shape). Workspace: spax_workspace_bytes(SPAX_OP_TIERED_GEMV, d_out, d_in)
- * bytes, ZEROED BEFORE FIRST USE (it holds arrival counters that every completed call leaves
- * at zero; zero it again after a device error). Counts outside [0, d_in] or an index outside
- * [0, d_in) set *d_status = SPAX_ERR_INDEX; such a column contributes zero.
- * Calls that share a workspace must not run concurrently.
+ * bytes, ZEROED BEFORE FIRST USE: it holds the split-K partial sums as flagged words that every
+ * completed call leaves at zero (zero it again after a device error). The CTAs that split a row
+ * tile wait for one another's partial sums (a wait bounded at 1 s, then SPAX_ERR_TIMEOUT): the
+ * launch is one wave of at most one CTA per SM and expects its whole grid to be resident at
+ * once. Counts outside [0, d_in] or an index outside [0, d_in) set *d_status = SPAX_ERR_INDEX;
+ * such a column contributes zero. Calls that share a workspace must not run concurrently.
  */
 spax_status spax_tiered_gemv(const spax_packed* h_W, const float* d_x, const int32_t* d_full_idx,
                              const int32_t* d_approx_idx, const int32_t* d_counts, float* d_y,
@@ -226,11 +229,11 @@ spax_status spax_dense_gemv(const void* d_Wt, const float* d_x, float* d_y, int 
  * have no counterpart of this entry point; it is an interface convenience.
  * - The first call on each device (with that device current) looks up the array's device
  *   address and caches it; make that first call before any stream capture on that device.
- * - Shapes whose split plan needs more than the array holds (more than 4096 arrival counters,
- *   or partial sums beyond the rest of the 4 MiB; d_out up to about 1M rows on a 148-SM GPU)
- *   are rejected with SPAX_ERR_WORKSPACE before anything is launched.
- * - The array's arrival counters start at zero when the library loads and every completed
- *   call leaves them at zero; nothing for the caller to initialise.
+ * - Shapes whose split plan needs more partial sums than the array holds are rejected with
+ *   SPAX_ERR_WORKSPACE before anything is launched (none on a 148-SM GPU: a plan with splits
+ *   needs at most S * d_out * 8 <= 148 * 2048 * 8 bytes, and one without needs none).
+ * - The array starts at zero when the library loads and every completed call leaves it at zero;
+ *   nothing for the caller to initialise.
  * - There is ONE array per device for the whole process: calls on the same device that can
  *   overlap (other streams, other threads, concurrent graph branches) race on it and give
  *   wrong results. Serialise them.

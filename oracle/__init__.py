@@ -29,6 +29,7 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "spax_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "libspax_oracle.so")
+_LIB_OMP_PATH = os.path.join(_HERE, "libspax_oracle_omp.so")  # same source, OpenMP over rows
 
 FULL_BF16 = 0
 FULL_INT4 = 1
@@ -39,60 +40,83 @@ OK = 0
 ERR_NONFINITE = 5
 
 
-def build(force: bool = False) -> str:
-    """Compile the oracle with gcc (IEEE fp32 steps: no fast-math, no FMA contraction)."""
-    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
-        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+def build(force: bool = False, omp: bool = False) -> str:
+    """Compile the oracle with gcc (IEEE fp32 steps: no fast-math, no FMA contraction). omp=True
+    builds the multi-core variant of the same source (products split over row chunks)."""
+    path = _LIB_OMP_PATH if omp else _LIB_PATH
+    if force or not os.path.exists(path) or os.path.getmtime(path) < os.path.getmtime(_SRC):
+        tmp = path + f".tmp{os.getpid()}"
         subprocess.run(
             ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
-             "-Wall", "-o", tmp, _SRC, "-lm"],
+             "-Wall", "-Wno-unknown-pragmas"] + (["-fopenmp"] if omp else []) +
+            ["-o", tmp, _SRC, "-lm"],
             check=True,
         )
-        os.replace(tmp, _LIB_PATH)
-    return _LIB_PATH
+        os.replace(tmp, path)
+    return path
 
 
 _lib = None
+_lib_omp = None
+_use_omp = False
+
+
+def use_openmp(on: bool = True) -> int:
+    """Route the products through the OpenMP build (on) or the plain one (off); returns the
+    number of threads the products then use."""
+    global _use_omp
+    _use_omp = bool(on)
+    return int(_L().oracle_threads())
 
 
 def _L():
-    global _lib
+    global _lib, _lib_omp
+    if _use_omp:
+        if _lib_omp is None:
+            _lib_omp = _load(build(omp=True))
+        return _lib_omp
     if _lib is None:
-        lib = ctypes.CDLL(build())
-        P = ctypes.c_void_p
-        i32, i64, f32, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_double
-        lib.oracle_tiers.argtypes = [P, i32, i32, f32, f32, i32, i32, i32, i32, i32, P, P, P, P]
-        lib.oracle_tiers.restype = i32
-        lib.oracle_quant2_group.argtypes = [P, i32, P, P, P]
-        lib.oracle_quant4_group.argtypes = [P, i32, P, P]
-        lib.oracle_pack.argtypes = [P, i32, i32, i32, P, P]
-        lib.oracle_pack.restype = i32
-        lib.oracle_pack_column.argtypes = [P, i32, i32, i32, i32, P, P]
-        lib.oracle_pack_column.restype = i32
-        lib.oracle_full_col_bytes.argtypes = [i32, i32]
-        lib.oracle_full_col_bytes.restype = i64
-        lib.oracle_approx_col_bytes.argtypes = [i32]
-        lib.oracle_approx_col_bytes.restype = i64
-        lib.oracle_full_value.argtypes = [P, i32, i32]
-        lib.oracle_full_value.restype = f64
-        lib.oracle_approx_value.argtypes = [P, i32]
-        lib.oracle_approx_value.restype = f64
-        lib.oracle_tiered_gemv.argtypes = [P, P, i32, i32, i32, P, P, P, i32, P]
-        lib.oracle_tiered_gemv.restype = i32
-        lib.oracle_dense_gemv.argtypes = [P, i32, i32, P, P, i32, P]
-        lib.oracle_dense_gemv.restype = i32
-        lib.oracle_calibrate.argtypes = [P, i64, i32, i32, P]
-        lib.oracle_calibrate.restype = i32
-        lib.oracle_block_budgets.argtypes = [P, i32, f64, f64, f64, f64, P]
-        lib.oracle_block_budgets.restype = i32
-        lib.oracle_weight_bytes.argtypes = [i32, i32, i64, i64]
-        lib.oracle_weight_bytes.restype = ctypes.c_uint64
-        lib.oracle_f32_to_bf16.argtypes = [f32]
-        lib.oracle_f32_to_bf16.restype = ctypes.c_uint16
-        lib.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
-        lib.oracle_bf16_to_f32.restype = f32
-        _lib = lib
+        _lib = _load(build())
     return _lib
+
+
+def _load(path):
+    lib = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    i32, i64, f32, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_double
+    lib.oracle_tiers.argtypes = [P, i32, i32, f32, f32, i32, i32, i32, i32, i32, P, P, P, P]
+    lib.oracle_tiers.restype = i32
+    lib.oracle_quant2_group.argtypes = [P, i32, P, P, P]
+    lib.oracle_quant4_group.argtypes = [P, i32, P, P]
+    lib.oracle_pack.argtypes = [P, i32, i32, i32, P, P]
+    lib.oracle_pack.restype = i32
+    lib.oracle_pack_column.argtypes = [P, i32, i32, i32, i32, P, P]
+    lib.oracle_pack_column.restype = i32
+    lib.oracle_full_col_bytes.argtypes = [i32, i32]
+    lib.oracle_full_col_bytes.restype = i64
+    lib.oracle_approx_col_bytes.argtypes = [i32]
+    lib.oracle_approx_col_bytes.restype = i64
+    lib.oracle_full_value.argtypes = [P, i32, i32]
+    lib.oracle_full_value.restype = f64
+    lib.oracle_approx_value.argtypes = [P, i32]
+    lib.oracle_approx_value.restype = f64
+    lib.oracle_tiered_gemv.argtypes = [P, P, i32, i32, i32, P, P, P, i32, P]
+    lib.oracle_tiered_gemv.restype = i32
+    lib.oracle_dense_gemv.argtypes = [P, i32, i32, P, P, i32, P]
+    lib.oracle_dense_gemv.restype = i32
+    lib.oracle_calibrate.argtypes = [P, i64, i32, i32, P]
+    lib.oracle_calibrate.restype = i32
+    lib.oracle_block_budgets.argtypes = [P, i32, f64, f64, f64, f64, P]
+    lib.oracle_block_budgets.restype = i32
+    lib.oracle_weight_bytes.argtypes = [i32, i32, i64, i64]
+    lib.oracle_weight_bytes.restype = ctypes.c_uint64
+    lib.oracle_f32_to_bf16.argtypes = [f32]
+    lib.oracle_f32_to_bf16.restype = ctypes.c_uint16
+    lib.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
+    lib.oracle_bf16_to_f32.restype = f32
+    lib.oracle_threads.argtypes = []
+    lib.oracle_threads.restype = i32
+    return lib
 
 
 def _p(a: np.ndarray):

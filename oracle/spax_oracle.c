@@ -35,6 +35,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define OR_OK 0
 #define OR_ERR_ARG 1
@@ -370,15 +373,22 @@ int oracle_tiered_gemv(const uint8_t* full, const uint8_t* approx, int fmt, int 
   if (d_out < 128 || d_out % 128 != 0 || d_in < 1) return OR_ERR_SHAPE;
   int64_t fcb = oracle_full_col_bytes(d_out, fmt), acb = oracle_approx_col_bytes(d_out);
   int ny = rows ? n_rows : d_out;
-  for (int i = 0; i < ny; ++i) y[i] = 0.0;
-  for (int j = 0; j < d_in; ++j) {
-    if (tier[j] == 0) continue;
-    double xj = (double)x[j];
-    for (int i = 0; i < ny; ++i) {
-      int r = rows ? rows[i] : i;
-      double w = tier[j] == 2 ? oracle_full_value(full + fcb * j, fmt, r)
-                              : oracle_approx_value(approx + acb * j, r);
-      y[i] += xj * w;
+  /* Outputs in chunks of 256 rows, each chunk summing its columns in ascending j. The chunks are
+     independent: the multi-core build (OpenMP) hands them to threads; every y[i] is the same
+     sum in the same order either way. */
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int c0 = 0; c0 < ny; c0 += 256) {
+    int c1 = ny - c0 < 256 ? ny : c0 + 256;
+    for (int i = c0; i < c1; ++i) y[i] = 0.0;
+    for (int j = 0; j < d_in; ++j) {
+      if (tier[j] == 0) continue;
+      double xj = (double)x[j];
+      for (int i = c0; i < c1; ++i) {
+        int r = rows ? rows[i] : i;
+        double w = tier[j] == 2 ? oracle_full_value(full + fcb * j, fmt, r)
+                                : oracle_approx_value(approx + acb * j, r);
+        y[i] += xj * w;
+      }
     }
   }
   return OR_OK;
@@ -396,6 +406,15 @@ int oracle_dense_gemv(const uint16_t* W, int d_out, int d_in, const float* x, co
     y[i] = acc;
   }
   return OR_OK;
+}
+
+/* Threads the products use: 1 in the plain build, the OpenMP team size in the multi-core one. */
+int oracle_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
 }
 
 /* ------------------------------------------------------------------ calibration ----------- */

@@ -445,3 +445,24 @@ def test_weight_bytes_account(oracle_lib):
         assert oracle_lib.weight_bytes(d_out, 0, 0, 1) == oracle_lib.approx_col_bytes(d_out)
         assert oracle_lib.weight_bytes(d_out, 0, 1, 0) == oracle_lib.full_col_bytes(d_out, 0)
         assert oracle_lib.weight_bytes(d_out, 1, 1, 0) == oracle_lib.full_col_bytes(d_out, 1)
+
+
+def test_openmp_build_gives_the_same_products(oracle_lib):
+    # The multi-core build only hands independent row chunks to threads: every output is the
+    # same sum in the same order, so the two builds agree bit for bit (ragged chunk included).
+    d_out, d_in = 640, 300
+    W = synth.weight(d_out, d_in, 1, 40)
+    x = synth.laplace((d_in,), 1, 41).numpy()
+    tier = np.random.default_rng(10).integers(0, 3, d_in).astype(np.uint8)
+    rows = np.array([639, 0, 300, 257, 256, 255], np.int32)
+    for fmt in (0, 1):
+        full, approx = oracle_lib.pack(bf16_bits(W), fmt)
+        y1 = oracle_lib.tiered_gemv(full, approx, fmt, d_out, d_in, x, tier)
+        r1 = oracle_lib.tiered_gemv(full, approx, fmt, d_out, d_in, x, tier, rows)
+        try:
+            assert oracle_lib.use_openmp(True) >= 1
+            yn = oracle_lib.tiered_gemv(full, approx, fmt, d_out, d_in, x, tier)
+            rn = oracle_lib.tiered_gemv(full, approx, fmt, d_out, d_in, x, tier, rows)
+        finally:
+            oracle_lib.use_openmp(False)
+        assert np.array_equal(y1, yn) and np.array_equal(r1, rn) and np.array_equal(r1, y1[rows])

@@ -3,7 +3,7 @@ no workspace argument, no allocation) against spax_tiered_gemv, through the C AB
 
 Each case runs the fixed-scratch call twice in a row on fresh tokens and compares each result with
 the workspace entry point within the parity tolerance. Shapes of different split plans alternate,
-so the arrival counters left by one shape must serve the next. This file is collected last on
+so the partial-sum words one shape leaves at zero must serve the next. This file is collected last on
 purpose: it must pass in a fresh process and after every other GPU test.
 """
 import numpy as np
@@ -49,16 +49,20 @@ def test_fixed_scratch_matches_workspace_call(fmt):
             check_y(y_fx, y_ws, f"{gm.d_out}x{gm.d_in} call {call}")
 
 
-def test_fixed_scratch_rejects_oversized_plan():
-    # d_out = 2^20 rows: one split per row tile, partial sums of 4 MiB > the array's room
+def test_fixed_scratch_unsplit_plan_uses_no_scratch():
+    # d_out = 2^20 rows and one column: one split per row tile (512 tiles, more CTAs than SMs),
+    # so no partial sums at all; every row is written straight from its tile, y = x_0 * W[:, 0].
     d_out, d_in = 1 << 20, 1
     assert spax.spax_fixed_scratch_bytes() == 4 << 20
-    pm = spax.alloc_packed(d_out, d_in, 0)
-    x = torch.ones(d_in, dtype=torch.float32, device="cuda")
-    idx = torch.zeros(d_in, dtype=torch.int32, device="cuda")
-    counts = torch.tensor([1, 0, 0, 0], dtype=torch.int32, device="cuda")
-    y = torch.empty(d_out, dtype=torch.float32, device="cuda")
-    status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    with pytest.raises(spax.SpaxError) as e:
-        spax.spax_tiered_gemv_fixed_scratch(pm, x, idx, idx, counts, y, status)
-    assert e.value.status == spax.ERR_WORKSPACE
+    assert spax.spax_gemv_plan(spax.OP_TIERED_GEMV, d_out, d_in)[0] == 1
+    W = synth.weight(d_out, d_in, 3, 790, device="cuda")
+    gm = GpuMatrix(W, 0)
+    x = torch.full((d_in,), -1.75, dtype=torch.float32, device="cuda")
+    for kf, ka in [(1, 0), (0, 1), (0, 0)]:
+        y_ws, y_fx, st = _token(gm, x, spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka))
+        assert st == 0
+        assert np.array_equal(y_fx, y_ws)
+        if kf:
+            assert np.array_equal(y_fx, (-1.75 * W[:, 0].float()).cpu().numpy())
+        if kf + ka == 0:
+            assert np.all(y_fx == 0.0)

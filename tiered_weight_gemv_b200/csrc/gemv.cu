@@ -25,9 +25,12 @@
 //   * 2-bit and int4 codes become floats with one LOP3 each: the code is masked into the
 //     mantissa of a power-of-two constant C (value C + q exactly), multiplied by x_j*scale and
 //     the constant's contribution C*Σ x_j*scale is removed once per row at the end.
-//   * Warps' partial rows are combined in shared memory in a fixed order; split-K partials go to
-//     a workspace and the last CTA of each tile to arrive (arrival ticket: no CTA ever waits for
-//     another) sums the S partials in split order, so results are bit-reproducible.
+//   * Warps' partial rows are combined in shared memory in a fixed order. Split-K partials go to
+//     the workspace as 64-bit words that carry the value and a ready flag together (one
+//     single-copy-atomic store: no fence and no arrival counter on the critical path); each of
+//     the S CTAs of a tile then sums one slice of the tile's rows over the S splits in split
+//     order (bit-reproducible) and clears the words it read. The grid is one wave, so the CTAs
+//     that wait for one another are all resident; the wait is bounded (SPAX_ERR_TIMEOUT).
 #include "common.cuh"
 #include "internal.h"
 #include "select.cuh"
@@ -66,14 +69,11 @@ struct GemvParams {
   const int32_t* aidx;
   const int32_t* counts;
   float* y;
-  float* part;      // [S][d_out]
-  float* gpart;     // [NG][d_out]
-  uint32_t* gtick;  // [T][NG]
-  uint32_t* ttick;  // [T]
+  unsigned long long* part;  // [S][d_out] flagged partial sums, zero at rest
   int32_t* status;
   long long full_col_stride;    // bytes between full-pool columns
   long long approx_col_stride;  // bytes between approx-pool columns
-  int d_out, d_in, S, G, NG;
+  int d_out, d_in, S;
   // fused mask (masked GEMV only): the rule, the optional outputs, the staged-list bytes
   spax_mask_params prm;
   uint8_t* tier_out;
@@ -102,67 +102,29 @@ __device__ __forceinline__ uint32_t ld_stream16(const uint8_t* p) {
   return __ldcs(reinterpret_cast<const unsigned short*>(p));
 }
 
-// Fixed-order sum of `cnt` partial rows [r0, r0+rows) (row stride d_out), written to dst + r0.
-// The partials are cut into consecutive batches of kb, sized so that every thread of the CTA has
-// one item (a float4 of one batch) with all its loads in flight; the batch sums are then added in
-// batch order. The association depends only on cnt and rows, so the result is reproducible.
-template <int NT>
-__device__ void reduce_rows(const float* src, int cnt, int d_out, int r0, int rows, float* dst,
-                            int tid, float4* scratch /* [nb][rows/4] */) {
-  constexpr int kMaxBatch = 16;
-  const int n4 = rows >> 2;
-  int nb = max(1, NT / max(n4, 1));
-  const int kb = min(kMaxBatch, (cnt + nb - 1) / nb);
-  nb = (cnt + kb - 1) / kb;
-  const size_t stride4 = static_cast<size_t>(d_out) >> 2;
-  const float4* s4 = reinterpret_cast<const float4*>(src + r0);
-  for (int item = tid; item < n4 * nb; item += NT) {
-    const int i = item % n4, b = item / n4;
-    const int k0 = b * kb, kn = min(cnt - k0, kb);
-    float4 v[kMaxBatch];
-#pragma unroll
-    for (int k = 0; k < kMaxBatch; ++k)
-      if (k < kn) v[k] = __ldcg(s4 + (size_t)(k0 + k) * stride4 + i);
-    float4 acc = v[0];
-#pragma unroll
-    for (int k = 1; k < kMaxBatch; ++k)
-      if (k < kn) {
-        acc.x += v[k].x;
-        acc.y += v[k].y;
-        acc.z += v[k].z;
-        acc.w += v[k].w;
-      }
-    if (nb == 1)
-      reinterpret_cast<float4*>(dst + r0)[i] = acc;
-    else
-      scratch[b * n4 + i] = acc;
-  }
-  if (nb == 1) return;
-  __syncthreads();
-  for (int i = tid; i < n4; i += NT) {
-    float4 acc = scratch[i];
-    for (int b = 1; b < nb; ++b) {
-      const float4 v = scratch[b * n4 + i];
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
-    }
-    reinterpret_cast<float4*>(dst + r0)[i] = acc;
-  }
+// ---- flagged partial sums: (value bits | 1 << 32) per 64-bit word; 0 means "not written" ----
+__device__ __forceinline__ void st_ll4(unsigned long long* p, float4 v) {
+  const unsigned long long f = 1ull << 32;
+  asm volatile("st.relaxed.gpu.global.v2.b64 [%0], {%1, %2};" ::"l"(p),
+               "l"(f | __float_as_uint(v.x)), "l"(f | __float_as_uint(v.y))
+               : "memory");
+  asm volatile("st.relaxed.gpu.global.v2.b64 [%0], {%1, %2};" ::"l"(p + 2),
+               "l"(f | __float_as_uint(v.z)), "l"(f | __float_as_uint(v.w))
+               : "memory");
 }
-
-// Arrival ticket of a split-K group: after a CTA barrier (every thread's partial stores are done),
-// one thread adds 1 with acquire-release semantics at GPU scope. The release publishes the whole
-// CTA's stores (they happen before it through the barrier); the last arrival's acquire makes every
-// other CTA's partials visible to it (and, through the next barrier, to its threads). The last
-// arrival resets the counter for the next call.
-__device__ __forceinline__ bool ticket_last(uint32_t* t, uint32_t n) {
-  uint32_t old;
-  asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(old) : "l"(t) : "memory");
-  const bool last = old == n - 1;
-  if (last) *t = 0u;
-  return last;
+// The four words at p, when all four carry their flag.
+__device__ __forceinline__ bool ld_ll4(const unsigned long long* p, float4* v) {
+  unsigned long long a, b, c, d;
+  asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
+  asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(c), "=l"(d) : "l"(p + 2) : "memory");
+  if (((a & b & c & d) >> 32) == 0) return false;  // a flag is the word's only high bit
+  *v = make_float4(__uint_as_float((uint32_t)a), __uint_as_float((uint32_t)b),
+                   __uint_as_float((uint32_t)c), __uint_as_float((uint32_t)d));
+  return true;
+}
+__device__ __forceinline__ void clear_ll4(unsigned long long* p) {
+  asm volatile("st.relaxed.gpu.global.v2.b64 [%0], {%1, %1};" ::"l"(p), "l"(0ull) : "memory");
+  asm volatile("st.relaxed.gpu.global.v2.b64 [%0], {%1, %1};" ::"l"(p + 2), "l"(0ull) : "memory");
 }
 
 // Shared memory of the fused kernel ahead of the GEMV's own areas: the selection's scratch and
@@ -560,9 +522,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
     }
   }
   __syncthreads();
-
-  float* out_base = (S == 1) ? p.y : p.part + (size_t)split * p.d_out;
-  for (int i = tid; i < rows_here / 4; i += kGemvThreads) {
+  // rows 4i..4i+3 of the tile: the column groups' slots summed in group order
+  auto combined_rows = [&](int i) -> float4 {
     float4 v = reinterpret_cast<const float4*>(red + red_row(4 * i))[0];
 #pragma unroll
     for (int c = 1; c < CG; ++c) {
@@ -572,28 +533,70 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
       v.z += w.z;
       v.w += w.w;
     }
-    reinterpret_cast<float4*>(out_base + r0)[i] = v;
-  }
-  if (S == 1) return;
+    return v;
+  };
 
-  // ---- split-K: the last split of each group (then of the tile) to arrive sums in order ----
-  const int grp = split / p.G;
-  const int gbeg = grp * p.G;
-  const int gsz = min(p.G, S - gbeg);
-  float4* scratch = reinterpret_cast<float4*>(red);  // [nb][R/4]: at most 24 KB, fits the slots
+  if (S == 1) {  // no split: the tile's rows are final
+    for (int i = tid; i < rows_here / 4; i += kGemvThreads)
+      reinterpret_cast<float4*>(p.y + r0)[i] = combined_rows(i);
+    return;
+  }
+
+  // ---- split-K: publish this split's rows, then reduce one slice of the tile's rows ----
+  // Each partial value travels with its ready flag in one 64-bit word (single-copy atomic), so
+  // a reader that sees the flag sees the value: no fence, no counter, one trip through L2. The
+  // S CTAs of a tile (all resident: the grid is one wave) each sum rows [4 g_lo, 4 g_hi) of the
+  // tile over the S splits in split order (bit-reproducible) and clear the words they read, so
+  // every completed call leaves the partial area at zero.
+  unsigned long long* part = p.part + (size_t)split * p.d_out + r0;
+  for (int i = tid; i < rows_here / 4; i += kGemvThreads) st_ll4(part + 4 * i, combined_rows(i));
+  const int n4 = rows_here / 4;
+  const int c4 = (n4 + S - 1) / S;
+  const int g_lo = min(n4, split * c4), ng = min(n4, g_lo + c4) - g_lo;
+  const int pairs = ng * S;  // (row group, source split) items, <= 2 per thread
+  float4* sc = reinterpret_cast<float4*>(red);  // [S][c4]
+  __syncthreads();  // the combine area is dead: reuse it as the gather scratch
+  {
+    const int q0 = tid, q1 = tid + kGemvThreads;
+    const bool h0 = q0 < pairs, h1 = q1 < pairs;
+    unsigned long long* a0 = h0 ? p.part + (size_t)(q0 / ng) * p.d_out + r0 + 4 * (g_lo + q0 % ng) : nullptr;
+    unsigned long long* a1 = h1 ? p.part + (size_t)(q1 / ng) * p.d_out + r0 + 4 * (g_lo + q1 % ng) : nullptr;
+    bool need0 = h0, need1 = h1;
+    unsigned long long t0 = 0;
+    for (int it = 0; need0 || need1; ++it) {
+      float4 v;
+      if (need0 && ld_ll4(a0, &v)) {
+        sc[(q0 / ng) * c4 + q0 % ng] = v;
+        clear_ll4(a0);
+        need0 = false;
+      }
+      if (need1 && ld_ll4(a1, &v)) {
+        sc[(q1 / ng) * c4 + q1 % ng] = v;
+        clear_ll4(a1);
+        need1 = false;
+      }
+      if ((need0 || need1) && (it & 15) == 15) {  // bounded: a missing split is a library bug
+        const unsigned long long now = global_timer_ns();
+        if (t0 == 0) t0 = now;
+        else if (now - t0 > kWaitLimitNs) {
+          record_status(p.status, SPAX_ERR_TIMEOUT);
+          break;
+        }
+      }
+    }
+  }
   __syncthreads();
-  if (tid == 0) s_last = ticket_last(p.gtick + (size_t)tile * p.NG + grp, (uint32_t)gsz);
-  __syncthreads();
-  if (!s_last) return;
-  float* gdst = (p.NG == 1) ? p.y : p.gpart + (size_t)grp * p.d_out;
-  reduce_rows<kGemvThreads>(p.part + (size_t)gbeg * p.d_out, gsz, p.d_out, r0, rows_here, gdst,
-                            tid, scratch);
-  if (p.NG == 1) return;
-  __syncthreads();
-  if (tid == 0) s_last = ticket_last(p.ttick + tile, (uint32_t)p.NG);
-  __syncthreads();
-  if (!s_last) return;
-  reduce_rows<kGemvThreads>(p.gpart, p.NG, p.d_out, r0, rows_here, p.y, tid, scratch);
+  for (int g = tid; g < ng; g += kGemvThreads) {
+    float4 acc = sc[g];
+    for (int q = 1; q < S; ++q) {
+      const float4 v = sc[q * c4 + g];
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    reinterpret_cast<float4*>(p.y + r0)[g_lo + g] = acc;
+  }
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -602,8 +605,9 @@ bool make_gemv_plan(int d_out, int d_in, int full_fmt, int sm_count, GemvPlan* p
   if (d_out < 128 || d_out % 128 != 0 || d_in < 1 || sm_count < 1) return false;
   if (full_fmt != SPAX_FULL_BF16 && full_fmt != SPAX_FULL_INT4_G128) return false;
   GemvPlan pl;
-  // Smallest row tile that still leaves >= 8 splits per tile: the last CTA of a tile sums
-  // S x R partial values, so a small S*R keeps the reduction short.
+  // Smallest row tile that still leaves >= 8 splits per tile: many splits per tile spread each
+  // selected column over several CTAs, and a short tile keeps each CTA's slice of the split-K
+  // reduction (R / S rows) small.
   pl.R = 2048;
   for (int r = 512; r <= 1024; r *= 2) {
     if ((d_out + r - 1) / r <= sm_count / 8) {
@@ -615,27 +619,10 @@ bool make_gemv_plan(int d_out, int d_in, int full_fmt, int sm_count, GemvPlan* p
   pl.S = sm_count / pl.T;
   if (pl.S < 1) pl.S = 1;
   if (pl.S > d_in) pl.S = d_in;
-  if (pl.S > 1024) pl.S = 1024;  // keeps the reduction batches within the combine area
-  // one level (the last of the S splits sums them all) unless S is large
-  if (pl.S <= 48) {
-    pl.G = pl.S;
-  } else {
-    int g = 1;
-    while (g * g < pl.S) ++g;
-    pl.G = g;
-  }
-  pl.NG = (pl.S + pl.G - 1) / pl.G;
+  if (pl.S > 256) pl.S = 256;  // keeps a CTA's reduction items within two per thread
   auto al = [](size_t v) { return (v + 255) & ~size_t(255); };
-  size_t off = 0;
-  pl.off_part = off;
-  off += al(size_t(pl.S) * d_out * 4);
-  pl.off_gpart = off;
-  off += al(size_t(pl.NG > 1 ? pl.NG : 0) * d_out * 4);
-  pl.off_gtick = off;
-  off += al(size_t(pl.T) * pl.NG * 4);
-  pl.off_ttick = off;
-  off += al(size_t(pl.T) * 4);
-  pl.ws_bytes = off;
+  pl.off_part = 0;
+  pl.ws_bytes = pl.S > 1 ? al(size_t(pl.S) * d_out * 8) : 256;  // flagged 64-bit partials
   *plan = pl;
   return true;
 }
@@ -679,10 +666,7 @@ static GemvParams make_params(const GemvLaunch& a, const GemvPlan& pl) {
   gp.aidx = a.approx_idx;
   gp.counts = a.counts;
   gp.y = a.y;
-  gp.part = reinterpret_cast<float*>(ws + pl.off_part);
-  gp.gpart = reinterpret_cast<float*>(ws + pl.off_gpart);
-  gp.gtick = reinterpret_cast<uint32_t*>(ws + pl.off_gtick);
-  gp.ttick = reinterpret_cast<uint32_t*>(ws + pl.off_ttick);
+  gp.part = reinterpret_cast<unsigned long long*>(ws + pl.off_part);
   gp.status = a.status;
   gp.full_col_stride = a.full_fmt == SPAX_FULL_BF16 ? 2LL * a.d_out
                                                     : (long long)((a.d_out + 1023) / 1024) * 528;
@@ -690,8 +674,6 @@ static GemvParams make_params(const GemvLaunch& a, const GemvPlan& pl) {
   gp.d_out = a.d_out;
   gp.d_in = a.d_in;
   gp.S = pl.S;
-  gp.G = pl.G;
-  gp.NG = pl.NG;
   gp.list_bytes = 0;
   return gp;
 }

@@ -9,11 +9,12 @@
 
 namespace spax {
 
-// Split-K plan of one GEMV launch: grid (T row tiles) x (S column splits); the S partial sums of
-// a tile are reduced in groups of G consecutive splits (NG groups), then over the groups.
+// Split-K plan of one GEMV launch: grid (T row tiles of R rows) x (S column splits), one wave
+// (T * S <= SMs whenever S > 1). The S flagged partial rows of a tile live at off_part in the
+// workspace ([S][d_out] 64-bit words, zero at rest); ws_bytes is the workspace the launch needs.
 struct GemvPlan {
-  int R, T, S, G, NG;
-  size_t off_part, off_gpart, off_gtick, off_ttick, ws_bytes;
+  int R, T, S;
+  size_t off_part, ws_bytes;
 };
 
 int sm_count_current_device();  // cached per device; 0 on error

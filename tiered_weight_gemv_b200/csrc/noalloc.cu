@@ -8,14 +8,11 @@
 // and callers that must not make the allocator synchronise the device. The regular entry point
 // needs a caller-owned workspace; this one does not.
 //
-// Scratch layout (kFixedScratchBytes in total, 256-byte aligned):
-//   [0, kTicketBytes)                 arrival counters of the split-K reduction. They must be
-//                                     zero before a call; device globals start at zero when the
-//                                     library's module loads and every completed call leaves
-//                                     them at zero again. Nothing else ever writes this range,
-//                                     so shapes of different calls never disturb each other's
-//                                     counters.
-//   [kTicketBytes, kFixedScratchBytes) partial sums (no initial value needed).
+// Scratch layout (kFixedScratchBytes in total, 256-byte aligned): the flagged split-K partial
+// sums of the launch's plan from offset 0. A word is zero until a split publishes its value (the
+// value's bits and a ready flag in one 64-bit store); the CTA that sums it clears it again. Device
+// globals start at zero when the library's module loads and every completed call leaves the
+// words it used at zero, so calls of any shape find a clean array.
 #include <mutex>
 
 #include "common.cuh"
@@ -24,7 +21,6 @@
 namespace spax {
 
 constexpr size_t kFixedScratchBytes = size_t(4) << 20;  // 4 MiB per device
-constexpr size_t kTicketBytes = size_t(16) << 10;       // 4096 counters
 
 static __device__ __align__(256) uint8_t g_fixed_scratch[kFixedScratchBytes];
 
@@ -70,19 +66,7 @@ spax_status spax_tiered_gemv_fixed_scratch(const spax_packed* W, const float* x,
   if (sms < 1) return SPAX_ERR_CUDA;
   GemvPlan pl;
   if (!make_gemv_plan(W->d_out, W->d_in, W->full_fmt, sms, &pl)) return SPAX_ERR_SHAPE;
-  // Same plan, relocated: counters first (in their reserved range), partial sums after them.
-  auto al = [](size_t v) { return (v + 255) & ~size_t(255); };
-  const size_t gtick_bytes = al(size_t(pl.T) * pl.NG * 4);
-  const size_t tick_bytes = gtick_bytes + al(size_t(pl.T) * 4);
-  const size_t part_bytes = al(size_t(pl.S) * W->d_out * 4);
-  const size_t gpart_bytes = al(size_t(pl.NG > 1 ? pl.NG : 0) * W->d_out * 4);
-  if (tick_bytes > kTicketBytes || kTicketBytes + part_bytes + gpart_bytes > kFixedScratchBytes)
-    return SPAX_ERR_WORKSPACE;
-  pl.off_gtick = 0;
-  pl.off_ttick = gtick_bytes;
-  pl.off_part = kTicketBytes;
-  pl.off_gpart = kTicketBytes + part_bytes;
-  pl.ws_bytes = kTicketBytes + part_bytes + gpart_bytes;
+  if (pl.ws_bytes > kFixedScratchBytes) return SPAX_ERR_WORKSPACE;
   uint8_t* scratch = fixed_scratch_current_device();
   if (!scratch) return SPAX_ERR_CUDA;
   GemvLaunch a;

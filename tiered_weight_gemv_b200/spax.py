@@ -287,7 +287,7 @@ def spax_dense_gemv(Wt: torch.Tensor, x: torch.Tensor, y: torch.Tensor, d_out: i
 
 
 def alloc_workspace(op: int, d_out: int, d_in: int, device="cuda") -> torch.Tensor:
-    """A zeroed workspace (the GEMV's arrival counters must start at zero)."""
+    """A zeroed workspace (the GEMV's flagged partial sums must start at zero)."""
     n = spax_workspace_bytes(op, d_out, d_in)
     if n == 0:
         raise SpaxError("spax_workspace_bytes", ERR_SHAPE)
