@@ -313,26 +313,28 @@ __device__ __forceinline__ void select_boundaries(const spax_mask_params& prm, i
     const uint32_t p0 = sel0 ? S.sel[0][0] : kNoKey, p1 = sel1 ? S.sel[1][0] : kNoKey;
     ab0 = sel0 ? S.sel[0][1] : 0u;
     ab1 = sel1 ? S.sel[1][1] : 0u;
-    // ---- pass 2: bits 18..9 of the keys in the two bins, and each sub-bin's largest key ----
-    for (int q = tid; q < nq; q += kSelThreads) {
-      const uint4 v = kq[q];
+    // ---- pass 2: bits 18..9 of the keys in the two bins. One atomic per key of either bin
+    // (both boundaries in one bin share ha[0]); a warp whose keys all miss skips the atomics.
+    const bool same = p0 == p1;
+    for (int qb = tid - lane; qb < nq; qb += kSelThreads) {  // warp-uniform trip count
+      const int q = qb + lane;
+      const uint4 v = q < nq ? kq[q] : make_uint4(kNoKey, kNoKey, kNoKey, kNoKey);
       const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const uint32_t b = kk[e] >> 19;
-        if (b == p0 || b == p1) {
-          const uint32_t sb = (kk[e] >> 9) & 1023u;
-          if (b == p0) atomicAdd(&S.ha[0][sb], 1u);
-          if (b == p1) atomicAdd(&S.ha[1][sb], 1u);
-        }
+        const bool m = b == p0 || b == p1;
+        if (__any_sync(0xffffffffu, m) && m)
+          atomicAdd(&S.ha[b == p0 ? 0 : 1][(kk[e] >> 9) & 1023u], 1u);
       }
     }
     if (tid == 0 && pad) {  // padding zeros of the last quad
       if (p0 == 0u) atomicSub(&S.ha[0][0], pad);
-      if (p1 == 0u) atomicSub(&S.ha[1][0], pad);
+      else if (p1 == 0u) atomicSub(&S.ha[1][0], pad);
     }
     __syncthreads();
-    block_find_pair<1024>(S.ha[0], S.ha[1], sel0, sel1, K0, K1, ab0, ab1, p0, p1, 10, S);
+    block_find_pair<1024>(S.ha[0], same ? S.ha[0] : S.ha[1], sel0, sel1, K0, K1, ab0, ab1, p0, p1,
+                          10, S);
     // resolved here when rank K is the sub-bin's last key: then the whole sub-bin is in
     bool need0 = false, need1 = false;
     uint32_t q0 = kNoKey, q1 = kNoKey;
@@ -361,22 +363,25 @@ __device__ __forceinline__ void select_boundaries(const spax_mask_params& prm, i
     if (need0 || need1) {
       const uint32_t abA0 = S.sel[0][1], abA1 = S.sel[1][1];
       __syncthreads();  // S.sel is rewritten below
-      for (int q = tid; q < nq; q += kSelThreads) {
-        const uint4 v = kq[q];
+      const bool same2 = q0 == q1;
+      for (int qb = tid - lane; qb < nq; qb += kSelThreads) {  // warp-uniform trip count
+        const int q = qb + lane;
+        const uint4 v = q < nq ? kq[q] : make_uint4(kNoKey, kNoKey, kNoKey, kNoKey);
         const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const uint32_t b = kk[e] >> 9;
-          if (b == q0) atomicAdd(&S.hb[0][kk[e] & 511u], 1u);
-          if (b == q1) atomicAdd(&S.hb[1][kk[e] & 511u], 1u);
+          const bool m = b == q0 || b == q1;
+          if (__any_sync(0xffffffffu, m) && m) atomicAdd(&S.hb[b == q0 ? 0 : 1][kk[e] & 511u], 1u);
         }
       }
       if (tid == 0 && pad) {
         if (q0 == 0u) atomicSub(&S.hb[0][0], pad);
-        if (q1 == 0u) atomicSub(&S.hb[1][0], pad);
+        else if (q1 == 0u) atomicSub(&S.hb[1][0], pad);
       }
       __syncthreads();
-      block_find_pair<512>(S.hb[0], S.hb[1], need0, need1, K0, K1, abA0, abA1, q0, q1, 9, S);
+      block_find_pair<512>(S.hb[0], same2 ? S.hb[0] : S.hb[1], need0, need1, K0, K1, abA0, abA1, q0,
+                           q1, 9, S);
       if (need0) V0 = S.sel[0][0], ab0 = S.sel[0][1], cnt0 = S.sel[0][2];
       if (need1) V1 = S.sel[1][0], ab1 = S.sel[1][1], cnt1 = S.sel[1][2];
     }
