@@ -251,6 +251,7 @@ def run_gpu(args, rank, world, local):
             counts=torch.empty(n_tok, 4, dtype=torch.int32, device=dev),
             y=torch.empty(n_tok, d_out, dtype=torch.float32, device=dev),
             yd=torch.empty(n_tok, d_out, dtype=torch.float32, device=dev),
+            yc=torch.empty(n_tok, d_out, dtype=torch.float32, device=dev),
             status=torch.zeros(1, dtype=torch.int32, device=dev),
             ws=spax.alloc_workspace(spax.OP_TIERED_GEMV, d_out, d_in, device=dev),
             dws=spax.alloc_workspace(spax.OP_DENSE_GEMV, d_out, d_in, device=dev),
@@ -285,6 +286,21 @@ def run_gpu(args, rank, world, local):
                                       full_idx=b["fidx"][t], approx_idx=b["aidx"][t],
                                       counts=b["counts"][t], desc=b["desc"][t % n_rep])
 
+    def step_chained():
+        """The decoder layer's MLP chained on the device: down's input is formed inside its
+        launch from the tiered gate/up output, x = silu(g) * u (informational; the headline feeds
+        every site its prepared input so each site's parity stands alone)."""
+        for t in range(n_tok):
+            for name, d_out, d_in, _ in SEL:
+                b = buf[name]
+                if name == "down" and "gate_up" in buf:
+                    spax.spax_masked_gemv_swiglu(packed[name][t % n_rep], buf["gate_up"]["y"][t],
+                                                 b["prm"], b["yc"][t], b["status"], b["ws"],
+                                                 desc=b["desc"][t % n_rep])
+                else:
+                    spax.spax_masked_gemv(packed[name][t % n_rep], xs[name][t], b["prm"], b["y"][t],
+                                          b["status"], b["ws"], desc=b["desc"][t % n_rep])
+
     def step_dense(sites=None):
         for t in range(n_tok):
             for name, d_out, d_in, _ in SEL:
@@ -315,6 +331,7 @@ def run_gpu(args, rank, world, local):
     graphs["fused"] = capture(step_fused)
     graphs["tiered"] = capture(step_tiered)
     graphs["dense"] = capture(step_dense)
+    graphs["chained"] = capture(step_chained)
     for name, *_ in SEL:
         graphs["fused_" + name] = capture(step_fused, sites=[name])
         graphs["gemv_" + name] = capture(step_tiered, mask=False, gemv=True, sites=[name])
@@ -327,6 +344,7 @@ def run_gpu(args, rank, world, local):
         res["fused"] = max_over_ranks(time_graph(graphs["fused"], args.steps, args.warmup, stream))
         res["tiered"] = max_over_ranks(time_graph(graphs["tiered"], args.steps, args.warmup, stream))
         res["dense"] = max_over_ranks(time_graph(graphs["dense"], args.steps, args.warmup, stream))
+        res["chained"] = max_over_ranks(time_graph(graphs["chained"], args.steps, args.warmup, stream))
         for name, *_ in SEL:
             res["fused_" + name] = max_over_ranks(
                 time_graph(graphs["fused_" + name], args.steps, args.warmup, stream))
@@ -730,6 +748,9 @@ def main():
             "dense_effective_GBps": round(dense_bytes / (res["dense"] * 1e-3) / 1e9, 1),
             "speedup_vs_dense": round(dense / value, 3),
             "two_call_us_per_token_layer": round(two_call, 3),
+            "chained_us_per_token_layer": round(us_per_token_layer(res["chained"], args.tokens, world), 3),
+            "chained_note": "down fed from the tiered gate/up output in its own launch "
+                            "(spax_masked_gemv_swiglu); informational",
             "sites": sites,
             "fit_time_vs_bytes": {"tiered": fit_c0_bw([(v["masked_gemv_bytes_per_launch"], v["masked_gemv_us"]) for v in sites.values()]),
                                   "dense": fit_c0_bw([(2 * v["d_out"] * v["d_in"], v["dense_us"]) for v in sites.values()])},

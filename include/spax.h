@@ -212,6 +212,24 @@ spax_status spax_masked_gemv(const spax_packed* h_W, const float* d_x,
                              int32_t* d_status, void* d_ws, size_t ws_bytes, void* stream);
 
 /*
+ * spax_masked_gemv_swiglu — spax_masked_gemv whose activation is formed in the kernel from the
+ * gated-MLP pair before it: x_j = silu(g_j) * u_j with silu(g) = g / (1 + e^-g), for the down
+ * projection fed straight from the tiered gate/up output. Source: the same passages as
+ * spax_masked_gemv; the chained gate/up -> down step is the decoder layer around them.
+ * d_gu: fp32 [2 * d_in] (device) = [g_0 .. g_{d_in-1}, u_0 .. u_{d_in-1}], i.e. the y of a gate/up
+ * matrix packed as gate rows then up rows. x_j is computed in fp32 (IEEE divide and multiply, the
+ * library's expf) by one function wherever the kernel needs it, so the tier rule and the product
+ * see the same value. d_x_out: fp32 [d_in] (device) receives that x; may be NULL. Every other
+ * argument, output and rule as spax_masked_gemv; a non-finite x_j (from a non-finite g or u, or
+ * an overflowing product) is SPAX_ERR_NONFINITE.
+ */
+spax_status spax_masked_gemv_swiglu(const spax_packed* h_W, const float* d_gu,
+                                    const spax_mask_params* h_params, float* d_y, float* d_x_out,
+                                    uint8_t* d_tier, int32_t* d_full_idx, int32_t* d_approx_idx,
+                                    int32_t* d_counts, int32_t* d_status, void* d_ws,
+                                    size_t ws_bytes, void* stream);
+
+/*
  * spax_dense_gemv — the same-GPU dense baseline: y = W x over every column, read from the
  * bf16 full pool (W^T [d_in][d_out]) with the same kernel family as spax_tiered_gemv.
  * Source: eigenradar commentary (comparisons use dense decoding in the same weight format).

@@ -281,6 +281,15 @@ def block_budgets(sens, s, lam, lo=0.05, hi=0.95):
     return out
 
 
+def swiglu(g, u):
+    """Gated-MLP activation feeding the down projection, x_j = silu(g_j) * u_j with
+    silu(g) = g / (1 + e^-g), in fp64 (the Llama-2-7B block's MLP: down reads SiLU(gate x) times
+    (up x)). Written from the definition; the library forms the same x in fp32."""
+    g = np.asarray(g, np.float64)
+    u = np.asarray(u, np.float64)
+    return g / (1.0 + np.exp(-g)) * u
+
+
 def greedy_allocation(params, alpha, p_target, err, p_max=1.0, step_base="mean", max_steps=100000):
     """Block-wise greedy per-matrix sparsity (TopK-Guided, Appendix D and Table 4), written out
     step by step: every matrix m has step alpha * base / f_m (base = the mean parameter count, or

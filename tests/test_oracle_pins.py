@@ -466,3 +466,21 @@ def test_openmp_build_gives_the_same_products(oracle_lib):
         finally:
             oracle_lib.use_openmp(False)
         assert np.array_equal(y1, yn) and np.array_equal(r1, rn) and np.array_equal(r1, y1[rows])
+
+
+def test_swiglu_closed_forms(oracle_lib):
+    # silu(0) = 0; silu(g) - silu(-g) = g (sigma(g) + sigma(-g) = 1); silu(g) = g/2 (1 + tanh(g/2))
+    # (a different closed form of the same function); the gate scales linearly in u.
+    g = np.array([0.0, 1e-8, 0.3, -0.3, 1.0, -2.5, 7.0, -12.0, 30.0, -30.0])
+    ones = np.ones_like(g)
+    s = oracle_lib.swiglu(g, ones)
+    assert s[0] == 0.0
+    assert np.allclose(s - oracle_lib.swiglu(-g, ones), g, rtol=1e-14, atol=1e-14)
+    mid = np.abs(g) <= 8  # the tanh form cancels in the negative tail; there use g e^g / (1 + e^g)
+    assert np.allclose(s[mid], (g / 2 * (1 + np.tanh(g / 2)))[mid], rtol=1e-13, atol=1e-300)
+    assert np.allclose(s, g * np.exp(g) / (1 + np.exp(g)), rtol=1e-14, atol=1e-300)
+    u = np.linspace(-3, 3, g.size)
+    assert np.allclose(oracle_lib.swiglu(g, u), s * u, rtol=1e-15, atol=0)
+    # far tails: silu(g) -> g for large g, -> g e^g (tiny, negative) for very negative g
+    assert oracle_lib.swiglu(40.0, 1.0) == 40.0
+    assert -1e-15 < oracle_lib.swiglu(-40.0, 1.0) < 0.0

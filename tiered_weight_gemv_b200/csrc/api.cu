@@ -215,10 +215,11 @@ spax_status spax_tiered_gemv(const spax_packed* W, const float* x, const int32_t
                      W->d_out, W->d_in, status, ws, ws_bytes, stream, false);
 }
 
-spax_status spax_masked_gemv(const spax_packed* W, const float* x, const spax_mask_params* p,
-                             float* y, uint8_t* tier, int32_t* full_idx, int32_t* approx_idx,
-                             int32_t* counts, int32_t* status, void* ws, size_t ws_bytes,
-                             void* stream) {
+static spax_status masked_gemv_common(const spax_packed* W, const float* x, bool swiglu,
+                                      float* x_out, const spax_mask_params* p, float* y,
+                                      uint8_t* tier, int32_t* full_idx, int32_t* approx_idx,
+                                      int32_t* counts, int32_t* status, void* ws, size_t ws_bytes,
+                                      void* stream) {
   if (!W || !W->d_full || !W->d_approx || !x || !p || !y) return SPAX_ERR_ARG;
   if (W->full_fmt != SPAX_FULL_BF16 && W->full_fmt != SPAX_FULL_INT4_G128) return SPAX_ERR_ARG;
   if (W->d_out < 128 || W->d_out % 128 != 0 || W->d_in < 1) return SPAX_ERR_SHAPE;
@@ -248,8 +249,25 @@ spax_status spax_masked_gemv(const spax_packed* W, const float* x, const spax_ma
   a.d_in = W->d_in;
   a.full_fmt = W->full_fmt;
   a.dense = false;
-  return launch_status(launch_masked_gemv(a, q, tier, full_idx, approx_idx, counts, pl,
-                                          static_cast<cudaStream_t>(stream)));
+  return launch_status(launch_masked_gemv(a, q, swiglu, x_out, tier, full_idx, approx_idx, counts,
+                                          pl, static_cast<cudaStream_t>(stream)));
+}
+
+spax_status spax_masked_gemv(const spax_packed* W, const float* x, const spax_mask_params* p,
+                             float* y, uint8_t* tier, int32_t* full_idx, int32_t* approx_idx,
+                             int32_t* counts, int32_t* status, void* ws, size_t ws_bytes,
+                             void* stream) {
+  return masked_gemv_common(W, x, false, nullptr, p, y, tier, full_idx, approx_idx, counts, status,
+                            ws, ws_bytes, stream);
+}
+
+spax_status spax_masked_gemv_swiglu(const spax_packed* W, const float* gu,
+                                    const spax_mask_params* p, float* y, float* x_out,
+                                    uint8_t* tier, int32_t* full_idx, int32_t* approx_idx,
+                                    int32_t* counts, int32_t* status, void* ws, size_t ws_bytes,
+                                    void* stream) {
+  return masked_gemv_common(W, gu, true, x_out, p, y, tier, full_idx, approx_idx, counts, status,
+                            ws, ws_bytes, stream);
 }
 
 spax_status spax_dense_gemv(const void* Wt, const float* x, float* y, int d_out, int d_in,

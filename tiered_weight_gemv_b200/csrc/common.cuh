@@ -134,6 +134,12 @@ __device__ __forceinline__ f2 bf16x2_to_f2(uint32_t w) {
   return r;
 }
 
+// Gated-MLP activation x = silu(g) * u, silu(g) = g / (1 + e^-g), in fp32 with each step rounded
+// on its own (no contraction): the one definition every use of x in a kernel goes through.
+__device__ __forceinline__ float swiglu_x(float g, float u) {
+  return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
+}
+
 __device__ __forceinline__ void record_status(int32_t* status, int32_t code) {
   if (status) atomicCAS(status, 0, code);
 }

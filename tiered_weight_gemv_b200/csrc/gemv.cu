@@ -81,6 +81,8 @@ struct GemvParams {
   int32_t* aidx_out;
   int32_t* counts_out;
   int list_bytes;  // 0 for the list-driven kernels
+  int swiglu;      // fused only: x holds [g; u] and x_j = swiglu_x(g_j, u_j)
+  float* x_out;    // fused swiglu only: the token's x (lead CTA; may be null)
 };
 
 // Code -> float: (word & (mask << p)) | bits(C) is the float C + code, exactly, when C = 2^(23-p)
@@ -177,7 +179,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
     select_zero(sel);
     pdl_wait();
     pdl_launch_dependents();
-    select_fetch(p.x, p.d_in, keys);
+    if (p.swiglu)
+      select_fetch_swiglu(p.x, p.d_in, keys, tile == 0 && split == 0 ? p.x_out : nullptr);
+    else
+      select_fetch(p.x, p.d_in, keys);
     const uint32_t ts = __float_as_uint(p.prm.t_skip) & 0x7FFFFFFFu;
     const uint32_t tf = __float_as_uint(p.prm.t_full) & 0x7FFFFFFFu;
     uint32_t n1, n2;
@@ -261,6 +266,15 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
   // 2-bit Σ x*scale and Σ x*min, int4 Σ x*scale (reduced over the warp at the end)
   float sA[4] = {0.f, 0.f, 0.f, 0.f}, bA[4] = {0.f, 0.f, 0.f, 0.f}, s4[4] = {0.f, 0.f, 0.f, 0.f};
 
+  // x_j of a selected column (the fused swiglu kernel forms it from g_j and u_j again, with the
+  // same function the selection used)
+  auto xval = [&](int col) -> float {
+    if constexpr (FUSED) {
+      if (p.swiglu) return swiglu_x(__ldg(p.x + col), __ldg(p.x + p.d_in + col));
+    }
+    return __ldg(p.x + col);
+  };
+
   // Column of local position i of this split's approximate / full list (in the current chunk):
   // the fused kernel reads its staged lists directly, the list-driven one its metadata arrays.
   auto colA = [&](int i) -> int {
@@ -288,7 +302,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
     float xk = 0.f;
     if (lane < nb) {
       const int col = colA(cg + CG * (k0 + lane));
-      xk = col >= 0 ? __ldg(p.x + col) : 0.f;  // an invalid column contributes zero
+      xk = col >= 0 ? xval(col) : 0.f;  // an invalid column contributes zero
     }
 #pragma unroll
     for (int t = 0; t < kChunks2; ++t)
@@ -378,7 +392,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
 #pragma unroll
         for (int u = 0; u < U; ++u) {
           int col = u < nfb ? colF(cg + CG * (kf + u)) : -1;
-          xf[u] = col >= 0 ? __ldg(p.x + col) : 0.f;
+          xf[u] = col >= 0 ? xval(col) : 0.f;
           const uint8_t* src = p.full + max(col, 0) * p.full_col_stride + off_full;
           w0[u] = (u < nfb && v0) ? ld_stream128(src) : make_uint4(0u, 0u, 0u, 0u);
           w1[u] = (u < nfb && v1) ? ld_stream128(src + 512) : make_uint4(0u, 0u, 0u, 0u);
@@ -437,7 +451,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
         float xk = 0.f;
         if (lane < nb) {
           const int col = colF(cg + CG * (kf + lane));
-          xk = col >= 0 ? __ldg(p.x + col) : 0.f;
+          xk = col >= 0 ? xval(col) : 0.f;
         }
 #pragma unroll
         for (int t = 0; t < 9; ++t)
@@ -686,11 +700,14 @@ cudaError_t launch_gemv(const GemvLaunch& a, const GemvPlan& pl, cudaStream_t st
   return launch_r<SPAX_FULL_INT4_G128, false, false>(gp, pl, smem, stream);
 }
 
-cudaError_t launch_masked_gemv(const GemvLaunch& a, const spax_mask_params& prm, uint8_t* tier,
-                               int32_t* full_idx, int32_t* approx_idx, int32_t* counts,
-                               const GemvPlan& pl, cudaStream_t stream) {
+cudaError_t launch_masked_gemv(const GemvLaunch& a, const spax_mask_params& prm, bool swiglu,
+                               float* x_out, uint8_t* tier, int32_t* full_idx,
+                               int32_t* approx_idx, int32_t* counts, const GemvPlan& pl,
+                               cudaStream_t stream) {
   GemvParams gp = make_params(a, pl);
   gp.prm = prm;
+  gp.swiglu = swiglu ? 1 : 0;
+  gp.x_out = swiglu ? x_out : nullptr;
   gp.tier_out = tier;
   gp.fidx_out = full_idx;
   gp.aidx_out = approx_idx;

@@ -36,9 +36,11 @@ struct GemvLaunch {
 cudaError_t launch_gemv(const GemvLaunch& a, const GemvPlan& plan, cudaStream_t stream);
 // The mask and the GEMV in one launch (every CTA computes the token's lists itself); the tier,
 // list and count outputs may be null. Shared memory it needs for a plan and d_in.
-cudaError_t launch_masked_gemv(const GemvLaunch& a, const spax_mask_params& prm, uint8_t* tier,
-                               int32_t* full_idx, int32_t* approx_idx, int32_t* counts,
-                               const GemvPlan& plan, cudaStream_t stream);
+// swiglu: a.x holds [g; u] (2 * d_in) and x_j = silu(g_j) * u_j (written to x_out when set).
+cudaError_t launch_masked_gemv(const GemvLaunch& a, const spax_mask_params& prm, bool swiglu,
+                               float* x_out, uint8_t* tier, int32_t* full_idx,
+                               int32_t* approx_idx, int32_t* counts, const GemvPlan& plan,
+                               cudaStream_t stream);
 size_t masked_gemv_smem_bytes(const GemvPlan& plan, int d_in);
 
 cudaError_t launch_mask(const float* x, int d_in, const spax_mask_params& p, uint8_t* tier,

@@ -107,6 +107,45 @@ __device__ __forceinline__ void select_fetch(const float* __restrict__ x, int d,
   __syncthreads();
 }
 
+// x_j = swiglu_x(g_j, u_j) from gu = [g; u] (2 d values) -> keys[] as raw fp32 bits, the tail
+// of the last quad zero; x_out (may be null) receives x. Ends with a barrier.
+__device__ __forceinline__ void select_fetch_swiglu(const float* __restrict__ gu, int d,
+                                                    uint32_t* __restrict__ keys,
+                                                    float* __restrict__ x_out) {
+  const int tid = threadIdx.x;
+  const float* g = gu;
+  const float* u = gu + d;
+  const bool vec = ((reinterpret_cast<uintptr_t>(g) | reinterpret_cast<uintptr_t>(u) |
+                     reinterpret_cast<uintptr_t>(x_out)) & 15u) == 0;
+  const int nfull = d >> 2;
+  if (vec) {
+    for (int q = tid; q < nfull; q += kSelThreads) {
+      const float4 a = __ldg(reinterpret_cast<const float4*>(g) + q);
+      const float4 b = __ldg(reinterpret_cast<const float4*>(u) + q);
+      const float4 v = make_float4(swiglu_x(a.x, b.x), swiglu_x(a.y, b.y), swiglu_x(a.z, b.z),
+                                   swiglu_x(a.w, b.w));
+      reinterpret_cast<float4*>(keys)[q] = v;
+      if (x_out) reinterpret_cast<float4*>(x_out)[q] = v;
+    }
+  } else {
+    for (int j = tid; j < 4 * nfull; j += kSelThreads) {
+      const float v = swiglu_x(__ldg(g + j), __ldg(u + j));
+      keys[j] = __float_as_uint(v);
+      if (x_out) x_out[j] = v;
+    }
+  }
+  if (tid < 4 && (d & 3)) {
+    const int j = 4 * nfull + tid;
+    float v = 0.f;
+    if (j < d) {
+      v = swiglu_x(__ldg(g + j), __ldg(u + j));
+      if (x_out) x_out[j] = v;
+    }
+    keys[j] = j < d ? __float_as_uint(v) : 0u;
+  }
+  __syncthreads();
+}
+
 // Pass 1: |x| keys written back, the threshold counts, the non-finite flag and (mode != 0) the
 // 12-bit histogram. mode: 0 threshold, 1 TopK, 2 guided. Ends with a barrier; n1, n2 and bad
 // are identical in every thread.

@@ -60,6 +60,8 @@ _SIGS = {
     "spax_dense_gemv": ([_P, _P, _P, _I, _I, _P, _P, _Z, _P], _I),
     "spax_masked_gemv": ([ctypes.POINTER(spax_packed), _P, ctypes.POINTER(spax_mask_params), _P,
                           _P, _P, _P, _P, _P, _P, _Z, _P], _I),
+    "spax_masked_gemv_swiglu": ([ctypes.POINTER(spax_packed), _P, ctypes.POINTER(spax_mask_params),
+                                 _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P], _I),
     "spax_tiered_gemv_fixed_scratch": ([ctypes.POINTER(spax_packed), _P, _P, _P, _P, _P, _P, _P],
                                        _I),
     "spax_fixed_scratch_bytes": ([], _Z),
@@ -256,6 +258,27 @@ def spax_masked_gemv(W: PackedMatrix, x: torch.Tensor, params: spax_mask_params,
         _dev(full_idx, torch.int32, "full_idx"), _dev(approx_idx, torch.int32, "approx_idx"),
         _dev(counts, torch.int32, "counts"), _dev(status, torch.int32, "status"),
         _dev(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def spax_masked_gemv_swiglu(W: PackedMatrix, gu: torch.Tensor, params: spax_mask_params,
+                            y: torch.Tensor, status: torch.Tensor, ws: torch.Tensor, x_out=None,
+                            tier=None, full_idx=None, approx_idx=None, counts=None, stream=None,
+                            desc=None) -> None:
+    """spax_masked_gemv on x = silu(g) * u formed in the kernel from gu = [g; u] (2 * d_in)."""
+    if gu.numel() != 2 * W.d_in or y.numel() != W.d_out:
+        raise ValueError("gu / y sizes do not match W")
+    for t, n in ((x_out, W.d_in), (tier, W.d_in), (full_idx, W.d_in), (approx_idx, W.d_in),
+                 (counts, 4)):
+        if t is not None and t.numel() < n:
+            raise ValueError("output too small")
+    d = W.desc() if desc is None else desc
+    _check("spax_masked_gemv_swiglu", _lib.spax_masked_gemv_swiglu(
+        ctypes.byref(d), _dev(gu, torch.float32, "gu"), ctypes.byref(params),
+        _dev(y, torch.float32, "y"), _dev(x_out, torch.float32, "x_out"),
+        _dev(tier, torch.uint8, "tier"), _dev(full_idx, torch.int32, "full_idx"),
+        _dev(approx_idx, torch.int32, "approx_idx"), _dev(counts, torch.int32, "counts"),
+        _dev(status, torch.int32, "status"), _dev(ws, None, "ws"),
+        ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def spax_tiered_gemv_fixed_scratch(W: PackedMatrix, x: torch.Tensor, full_idx: torch.Tensor,
