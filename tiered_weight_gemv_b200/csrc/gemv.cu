@@ -132,7 +132,7 @@ __device__ __forceinline__ void clear_ll4(unsigned long long* p) {
 // Shared memory of the fused kernel ahead of the GEMV's own areas: the selection's scratch and
 // keys share space with the combine and staging areas (they are dead before the GEMV starts).
 __host__ __device__ inline size_t fused_select_bytes(int d) {
-  return (sizeof(SelectSmem) + 15) / 16 * 16 + select_keys_bytes(d);
+  return (sizeof(SelectSmem) + 15) / 16 * 16 + select_keys_bytes(d) + (size_t(d) + 3) / 4 / 16 * 16 + 16;
 }
 
 // FUSED: the kernel first runs the tier rule on x itself (select.cuh: every CTA computes the
@@ -187,7 +187,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
     const uint32_t tf = __float_as_uint(p.prm.t_full) & 0x7FFFFFFFu;
     uint32_t n1, n2;
     bool bad;
-    select_pass1(p.prm.mode, p.d_in, ts, tf, keys, sel, &n1, &n2, &bad);
+    uint8_t* sgn = reinterpret_cast<uint8_t*>(keys) + select_keys_bytes(p.d_in);
+    select_pass1(p.prm.mode, p.d_in, ts, tf, keys, sel, &n1, &n2, &bad, sgn);
     const bool lead = tile == 0 && split == 0;
     if (bad) {  // non-finite x: every tier 0, empty lists, y = 0
       Kf = 0;
@@ -221,6 +222,15 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
           p.counts_out[3] = p.prm.mode == SPAX_MASK_TOPK ? 0 : (int32_t)n2;
         }
       }
+      // signed x of this split's first kGemvMeta positions of each list, kept in the metadata
+      // arrays (idle in this kernel) for the product: no reload, no recomputation
+      const int nfl = min(kGemvMeta, Kf > split ? (Kf - split + S - 1) / S : 0);
+      const int nal = min(kGemvMeta, Ka > split ? (Ka - split + S - 1) / S : 0);
+      for (int i = tid; i < nfl; i += kGemvThreads)
+        reinterpret_cast<float*>(meta_col_f)[i] = select_signed_x(keys, sgn, list[split + S * i]);
+      for (int i = tid; i < nal; i += kGemvThreads)
+        reinterpret_cast<float*>(meta_col_a)[i] = select_signed_x(keys, sgn, list[a0 + split + S * i]);
+      __syncthreads();  // the keys are dead from here: the GEMV's staging areas reuse them
     }
   } else {
     pdl_wait();
@@ -275,6 +285,21 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
     return __ldg(p.x + col);
   };
 
+  // x of local position i of this split's approximate / full list: the fused kernel's stash
+  // (first kGemvMeta positions), else x of the column
+  auto xA = [&](int i, int col) -> float {
+    if constexpr (FUSED) {
+      if (i < kGemvMeta) return reinterpret_cast<const float*>(meta_col_a)[i];
+    }
+    return xval(col);
+  };
+  auto xF = [&](int i, int col) -> float {
+    if constexpr (FUSED) {
+      if (i < kGemvMeta) return reinterpret_cast<const float*>(meta_col_f)[i];
+    }
+    return xval(col);
+  };
+
   // Column of local position i of this split's approximate / full list (in the current chunk):
   // the fused kernel reads its staged lists directly, the list-driven one its metadata arrays.
   auto colA = [&](int i) -> int {
@@ -301,8 +326,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
     }
     float xk = 0.f;
     if (lane < nb) {
-      const int col = colA(cg + CG * (k0 + lane));
-      xk = col >= 0 ? xval(col) : 0.f;  // an invalid column contributes zero
+      const int i = cg + CG * (k0 + lane), col = colA(i);
+      xk = col >= 0 ? xA(i, col) : 0.f;  // an invalid column contributes zero
     }
 #pragma unroll
     for (int t = 0; t < kChunks2; ++t)
@@ -391,8 +416,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
         float xf[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-          int col = u < nfb ? colF(cg + CG * (kf + u)) : -1;
-          xf[u] = col >= 0 ? xval(col) : 0.f;
+          const int i = cg + CG * (kf + u);
+          const int col = u < nfb ? colF(i) : -1;
+          xf[u] = col >= 0 ? xF(i, col) : 0.f;
           const uint8_t* src = p.full + max(col, 0) * p.full_col_stride + off_full;
           w0[u] = (u < nfb && v0) ? ld_stream128(src) : make_uint4(0u, 0u, 0u, 0u);
           w1[u] = (u < nfb && v1) ? ld_stream128(src + 512) : make_uint4(0u, 0u, 0u, 0u);
@@ -450,8 +476,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
         }
         float xk = 0.f;
         if (lane < nb) {
-          const int col = colF(cg + CG * (kf + lane));
-          xk = col >= 0 ? xval(col) : 0.f;
+          const int i = cg + CG * (kf + lane), col = colF(i);
+          xk = col >= 0 ? xF(i, col) : 0.f;
         }
 #pragma unroll
         for (int t = 0; t < 9; ++t)

@@ -118,14 +118,28 @@ __device__ __forceinline__ void select_fetch_swiglu(const float* __restrict__ gu
   const bool vec = ((reinterpret_cast<uintptr_t>(g) | reinterpret_cast<uintptr_t>(u) |
                      reinterpret_cast<uintptr_t>(x_out)) & 15u) == 0;
   const int nfull = d >> 2;
-  if (vec) {
-    for (int q = tid; q < nfull; q += kSelThreads) {
-      const float4 a = __ldg(reinterpret_cast<const float4*>(g) + q);
-      const float4 b = __ldg(reinterpret_cast<const float4*>(u) + q);
-      const float4 v = make_float4(swiglu_x(a.x, b.x), swiglu_x(a.y, b.y), swiglu_x(a.z, b.z),
-                                   swiglu_x(a.w, b.w));
-      reinterpret_cast<float4*>(keys)[q] = v;
-      if (x_out) reinterpret_cast<float4*>(x_out)[q] = v;
+  if (vec) {  // batches of kB quads per thread: all loads of a batch in flight together
+    constexpr int kB = 6;
+    for (int q0 = tid; q0 < nfull; q0 += kB * kSelThreads) {
+      float4 a[kB], b[kB];
+#pragma unroll
+      for (int k = 0; k < kB; ++k) {
+        const int q = q0 + k * kSelThreads;
+        if (q < nfull) {
+          a[k] = __ldg(reinterpret_cast<const float4*>(g) + q);
+          b[k] = __ldg(reinterpret_cast<const float4*>(u) + q);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < kB; ++k) {
+        const int q = q0 + k * kSelThreads;
+        if (q < nfull) {
+          const float4 v = make_float4(swiglu_x(a[k].x, b[k].x), swiglu_x(a[k].y, b[k].y),
+                                       swiglu_x(a[k].z, b[k].z), swiglu_x(a[k].w, b[k].w));
+          reinterpret_cast<float4*>(keys)[q] = v;
+          if (x_out) reinterpret_cast<float4*>(x_out)[q] = v;
+        }
+      }
     }
   } else {
     for (int j = tid; j < 4 * nfull; j += kSelThreads) {
@@ -146,12 +160,22 @@ __device__ __forceinline__ void select_fetch_swiglu(const float* __restrict__ gu
   __syncthreads();
 }
 
+// Sign bits of quad q's four x values (bit e for x[4q + e]), for select_signed_x.
+__device__ __forceinline__ uint8_t quad_signs(uint4 v) {
+  return (uint8_t)((v.x >> 31) | ((v.y >> 31) << 1) | ((v.z >> 31) << 2) | ((v.w >> 31) << 3));
+}
+// x_j again from its |x| key and the sign bytes pass 1 kept.
+__device__ __forceinline__ float select_signed_x(const uint32_t* keys, const uint8_t* sgn, int j) {
+  return __uint_as_float(keys[j] | ((uint32_t)(sgn[j >> 2] >> (j & 3)) << 31));
+}
+
 // Pass 1: |x| keys written back, the threshold counts, the non-finite flag and (mode != 0) the
-// 12-bit histogram. mode: 0 threshold, 1 TopK, 2 guided. Ends with a barrier; n1, n2 and bad
-// are identical in every thread.
+// 12-bit histogram; sgn (may be null; (d + 3) / 4 bytes) keeps the signs. mode: 0 threshold,
+// 1 TopK, 2 guided. Ends with a barrier; n1, n2 and bad are identical in every thread.
 __device__ __forceinline__ void select_pass1(int mode, int d, uint32_t ts, uint32_t tf,
                                              uint32_t* __restrict__ keys, SelectSmem& S,
-                                             uint32_t* n1, uint32_t* n2, bool* bad) {
+                                             uint32_t* n1, uint32_t* n2, bool* bad,
+                                             uint8_t* __restrict__ sgn = nullptr) {
   const int tid = threadIdx.x, lane = tid & 31;
   const int nq = (d + 3) >> 2;
   uint4* kq = reinterpret_cast<uint4*>(keys);
@@ -159,6 +183,7 @@ __device__ __forceinline__ void select_pass1(int mode, int d, uint32_t ts, uint3
   if (mode == SPAX_MASK_TOPK) {
     for (int q = tid; q < nq; q += kSelThreads) {
       uint4 v = kq[q];
+      if (sgn) sgn[q] = quad_signs(v);
       v.x &= 0x7FFFFFFFu, v.y &= 0x7FFFFFFFu, v.z &= 0x7FFFFFFFu, v.w &= 0x7FFFFFFFu;
       atomicAdd(&S.hist[v.x >> 19], 1u);
       atomicAdd(&S.hist[v.y >> 19], 1u);
@@ -170,6 +195,7 @@ __device__ __forceinline__ void select_pass1(int mode, int d, uint32_t ts, uint3
     const bool hist = mode == SPAX_MASK_GUIDED;
     for (int q = tid; q < nq; q += kSelThreads) {
       uint4 v = kq[q];
+      if (sgn) sgn[q] = quad_signs(v);
       v.x &= 0x7FFFFFFFu, v.y &= 0x7FFFFFFFu, v.z &= 0x7FFFFFFFu, v.w &= 0x7FFFFFFFu;
       cs += (v.x < ts) + (v.y < ts) + (v.z < ts) + (v.w < ts);
       cf += (v.x < tf) + (v.y < tf) + (v.z < tf) + (v.w < tf);
