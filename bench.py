@@ -578,7 +578,7 @@ def fit_c0_bw(points):
 
 
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "tiered_gemv_traffic.json")
-GEMV_SOURCES = ["gemv.cu", "common.cuh", "internal.h"]
+GEMV_SOURCES = ["gemv.cu", "select.cuh", "common.cuh", "internal.h"]
 
 
 def gemv_source_hash() -> str:
