@@ -47,7 +47,8 @@ constexpr int kGemvU = 4;        // columns in flight per warp
 // so a warp keeps 2-4 KB in flight instead of a few bytes per lane.
 constexpr int kBatch2 = 16;                // 2-bit columns per staged batch
 constexpr int kBatch4 = 16;                // int4 columns per staged batch
-constexpr int kStageRecBytes = 16 * 272;   // = max(16 * 144, 16 * 272)
+constexpr int kStage2Bytes = 16 * 144;      // one batch of 2-bit records
+constexpr int kStageRecBytes = 2 * kStage2Bytes;  // two 2-bit batches (>= one int4 batch, 16 * 272)
 constexpr int kStageWarpBytes = kStageRecBytes + 16 * 16;  // + 4 coefficients per column
 
 template <int RG>
@@ -58,7 +59,7 @@ struct GemvCfg {
   static constexpr size_t kSmemBytes = size_t(2) * kGemvMeta * 4 + size_t(CG) * kSlotFloats * 4 +
                                        size_t(kGemvWarps) * kStageWarpBytes;
   static_assert(CG >= 4, "reduction scratch must fit the combine area");
-  static_assert(kBatch4 * 272 <= kStageRecBytes && kBatch2 * 144 <= kStageRecBytes, "staging");
+  static_assert(kBatch4 * 272 <= kStageRecBytes && 2 * kBatch2 * 144 <= kStageRecBytes, "staging");
 };
 
 struct GemvParams {
@@ -352,8 +353,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
   // 2-bit column k of the staged batch: 16 rows per word, row k at bits 2k. Rotations by 17 and
   // 25 bring rows 0-3 and 4-7 of an 8-row group to mantissa bits 15, 17, 19, 21: values 256+q,
   // 64+q, 16+q, 4+q.
-  auto decode_approx = [&](int k) {
-    const uint32_t rec = stage_s + 144 * k;
+  auto decode_approx = [&](int k, int buf = 0) {
+    const uint32_t rec = stage_s + kStage2Bytes * buf + 144 * k;
     const uint32_t q01 = lds32(rec + 2 * (lane & ~1)) >> (16 * (lane & 1));  // 2 bytes at 2*lane
     const uint32_t q11 = lds32(rec + 64 + 2 * (lane & ~1)) >> (16 * (lane & 1));
     const float c0 = __uint_as_float(lds32(coef_s + 16 * k + 4 * (lane / 16)));
@@ -368,6 +369,42 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
       acc[4 * b + 2] = ffma2(f2{code_f(rc, 3u << 15, 0x43800000u), code_f(rc, 3u << 17, 0x42800000u)}, c2, acc[4 * b + 2]);
       acc[4 * b + 3] = ffma2(f2{code_f(rc, 3u << 19, 0x41800000u), code_f(rc, 3u << 21, 0x40800000u)}, c2, acc[4 * b + 3]);
     }
+  };
+
+  // Asynchronous form for the bf16 path: the records of a batch are copied to staging buffer
+  // buf by cp.async (no registers held) while the warp streams bf16 columns and decodes the
+  // previous batch; stage_ready waits for them and prepares the batch's coefficients.
+  auto stage_issue = [&](int k0, int nb, int buf) {
+    __syncwarp();  // every lane is done with what this buffer held
+    const uint32_t dst = stage_s + kStage2Bytes * buf;
+    for (int q = lane; q < nb * 9; q += 32) {
+      const int k = q / 9, piece = q - 9 * k;
+      const int col = max(colA(cg + CG * (k0 + k)), 0);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + 16 * q),
+                   "l"(p.approx + col * p.approx_col_stride + off_approx + 16 * piece)
+                   : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  auto stage_ready = [&](int k0, int nb, int buf) {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncwarp();
+    if (lane < nb) {
+      const int i = cg + CG * (k0 + lane), col = colA(i);
+      const float xk = col >= 0 ? xA(i, col) : 0.f;  // an invalid column contributes zero
+      const uint4 sm = lds128(stage_s + kStage2Bytes * buf + 144 * lane + 128);
+      const uint32_t w[4] = {sm.x, sm.y, sm.z, sm.w};
+      float c[4];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        c[g] = xk * __uint_as_float(w[g] << 16);
+        sA[g] += c[g];
+        bA[g] = fmaf(xk, __uint_as_float(w[g] & 0xFFFF0000u), bA[g]);
+      }
+      asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(coef_s + 16 * lane), "f"(c[0]),
+                   "f"(c[1]), "f"(c[2]), "f"(c[3]));
+    }
+    __syncwarp();
   };
 
   for (int ch = 0; ch < nchunks; ++ch) {
@@ -409,7 +446,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
       // bf16 batches of U columns interleaved with 2-bit columns, so the dequant work of the
       // 2-bit tier runs while the bf16 loads are in flight
       const int per_it = nFw > 0 ? (nAw * U + nFw - 1) / nFw : nAw;
-      int ka = 0, kf = 0, sbeg = 0, send = 0;
+      int ka = 0, kf = 0, sbeg = 0, send = 0, buf = 0;
+      if (nAw > 0) stage_issue(0, min(kBatch2, nAw), 0);  // on its way before the first bf16 loads
       while (ka < nAw || kf < nFw) {
         const int nfb = max(0, min(U, nFw - kf));
         uint4 w0[U], w1[U];
@@ -425,14 +463,16 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
         }
         int todo = (kf + nfb < nFw) ? min(per_it, nAw - ka) : nAw - ka;
         while (todo > 0) {
-          if (ka == send) {
+          if (ka == send) {  // the batch at ka is in flight: wait, then send the next one
             sbeg = ka;
             send = ka + min(kBatch2, nAw - ka);
-            stage_approx(sbeg, send - sbeg);
+            buf = (sbeg / kBatch2) & 1;
+            stage_ready(sbeg, send - sbeg, buf);
+            if (send < nAw) stage_issue(send, min(kBatch2, nAw - send), buf ^ 1);
           }
           const int n = min(todo, send - ka);
 #pragma unroll 2
-          for (int k = ka; k < ka + n; ++k) decode_approx(k - sbeg);
+          for (int k = ka; k < ka + n; ++k) decode_approx(k - sbeg, buf);
           ka += n;
           todo -= n;
         }
