@@ -142,6 +142,17 @@ spax_status spax_pack_weights(const void* d_W, int d_out, int d_in, int full_fmt
                               void* d_approx, void* stream);
 
 /*
+ * spax_column_norms — offline: the Euclidean norm of every column of W, for the WINA score.
+ * Source: TopK-Guided §C.1 (WINA's per-element score of a column: the activation's magnitude
+ * times the column's norm) and §1 (WINA's fixed-count TopK rule).
+ * norm_j = fp32(sqrt(Σ_r W[r][j]^2)), the sum in fp64 in row order (each bf16 square is exact
+ * in fp64), sqrt correctly rounded, then rounded to fp32: one fixed definition, so every caller
+ * that follows it gets the same bits. d_W: row-major [d_out][d_in] bf16 (device); d_norms: fp32
+ * [d_in] (device), fully written. SPAX_ERR_SHAPE if d_out or d_in < 1.
+ */
+spax_status spax_column_norms(const void* d_W, int d_out, int d_in, float* d_norms, void* stream);
+
+/*
  * spax_calibrate_thresholds — offline: the calibrated |x| thresholds of the threshold and
  * guided rules (TopK-Guided §2.1 "calibrated threshold", §2.2 calibration pass).
  * Pools the M = n_tok * d_in values |x| of d_calib_x (row-major [n_tok][d_in] fp32) and, for
@@ -223,6 +234,22 @@ spax_status spax_masked_gemv(const spax_packed* h_W, const float* d_x,
  * argument, output and rule as spax_masked_gemv; a non-finite x_j (from a non-finite g or u, or
  * an overflowing product) is SPAX_ERR_NONFINITE.
  */
+/*
+ * spax_masked_gemv_wina — spax_masked_gemv whose rule ranks columns by the WINA score
+ * s_j = |x_j| * norm_j instead of |x_j|. Source: TopK-Guided §1 (WINA's TopK rule) and §C.1
+ * (its per-element score: activation magnitude times the column norm).
+ * d_norms: fp32 [d_in] (device), as spax_column_norms writes them. The score is one correctly
+ * rounded fp32 product; every rule (threshold, TopK, guided) and tie order of spax_build_mask
+ * then applies to s in place of |x| (thresholds are on s). The product still uses x. A
+ * non-finite score is SPAX_ERR_NONFINITE. Every other argument, output and rule as
+ * spax_masked_gemv.
+ */
+spax_status spax_masked_gemv_wina(const spax_packed* h_W, const float* d_x,
+                                  const float* d_norms, const spax_mask_params* h_params,
+                                  float* d_y, uint8_t* d_tier, int32_t* d_full_idx,
+                                  int32_t* d_approx_idx, int32_t* d_counts, int32_t* d_status,
+                                  void* d_ws, size_t ws_bytes, void* stream);
+
 spax_status spax_masked_gemv_swiglu(const spax_packed* h_W, const float* d_gu,
                                     const spax_mask_params* h_params, float* d_y, float* d_x_out,
                                     uint8_t* d_tier, int32_t* d_full_idx, int32_t* d_approx_idx,

@@ -114,6 +114,8 @@ def _load(path):
     lib.oracle_f32_to_bf16.restype = ctypes.c_uint16
     lib.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
     lib.oracle_bf16_to_f32.restype = f32
+    lib.oracle_column_norms.argtypes = [P, i32, i32, P]
+    lib.oracle_column_norms.restype = i32
     lib.oracle_threads.argtypes = []
     lib.oracle_threads.restype = i32
     return lib
@@ -279,6 +281,26 @@ def block_budgets(sens, s, lam, lo=0.05, hi=0.95):
     if st != OK:
         raise ValueError(f"oracle_block_budgets status {st}")
     return out
+
+
+def column_norms(W_bits):
+    """fp32 norm of every column of the row-major bf16 W (uint16 bits), for the WINA score
+    (TopK-Guided §C.1): fp64 sum of squares in row order, correctly rounded sqrt, then fp32."""
+    W = _c(W_bits, np.uint16)
+    d_out, d_in = W.shape
+    out = np.zeros(d_in, np.float32)
+    st = _L().oracle_column_norms(_p(W), d_out, d_in, _p(out))
+    if st != OK:
+        raise ValueError(f"oracle_column_norms status {st}")
+    return out
+
+
+def wina_scores(x, norms):
+    """WINA score s_j = |x_j| * norm_j, one IEEE fp32 product (TopK-Guided §1, §C.1); the tier rule
+    then ranks s in place of |x|."""
+    x = _c(x, np.float32)
+    norms = _c(norms, np.float32)
+    return (np.abs(x) * norms).astype(np.float32)
 
 
 def swiglu(g, u):

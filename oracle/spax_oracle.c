@@ -408,6 +408,25 @@ int oracle_dense_gemv(const uint16_t* W, int d_out, int d_in, const float* x, co
   return OR_OK;
 }
 
+/*
+ * Column norms for the WINA score [TKG §C.1: the per-element score of a column is the
+ * activation's magnitude times the column's norm]: norm_j = (float) sqrt(Σ_r W[r][j]^2), the
+ * squares (exact in fp64) summed in fp64 in row order, sqrt correctly rounded, one rounding to
+ * fp32.
+ */
+int oracle_column_norms(const uint16_t* W, int d_out, int d_in, float* norms) {
+  if (d_out < 1 || d_in < 1) return OR_ERR_SHAPE;
+  for (int j = 0; j < d_in; ++j) {
+    double acc = 0.0;
+    for (int r = 0; r < d_out; ++r) {
+      double w = (double)oracle_bf16_to_f32(W[(int64_t)r * d_in + j]);
+      acc += w * w;
+    }
+    norms[j] = (float)sqrt(acc);
+  }
+  return OR_OK;
+}
+
 /* Threads the products use: 1 in the plain build, the OpenMP team size in the multi-core one. */
 int oracle_threads(void) {
 #ifdef _OPENMP

@@ -484,3 +484,46 @@ def test_swiglu_closed_forms(oracle_lib):
     # far tails: silu(g) -> g for large g, -> g e^g (tiny, negative) for very negative g
     assert oracle_lib.swiglu(40.0, 1.0) == 40.0
     assert -1e-15 < oracle_lib.swiglu(-40.0, 1.0) < 0.0
+
+
+def test_column_norms_definition(oracle_lib):
+    # the definition written out in Python on a small matrix (fp64 sum in row order, sqrt, fp32)
+    rng = np.random.default_rng(21)
+    W = torch.tensor(rng.normal(0, 0.05, (37, 11)), dtype=torch.float32).to(torch.bfloat16)
+    Wb = bf16_bits(W)
+    n = oracle_lib.column_norms(Wb)
+    Wf = W.float().double().numpy()
+    for j in range(11):
+        acc = 0.0
+        for r in range(37):
+            acc += Wf[r, j] * Wf[r, j]
+        assert n[j] == np.float32(math.sqrt(acc))
+    # closed forms: a column of one value c has norm |c| sqrt(d_out); a zero column has norm 0
+    C = torch.zeros(64, 3, dtype=torch.bfloat16)
+    C[:, 0] = 0.375
+    C[:, 1] = -2.0
+    n = oracle_lib.column_norms(bf16_bits(C))
+    assert n[0] == np.float32(0.375 * 8.0) and n[1] == np.float32(16.0) and n[2] == 0.0
+
+
+def test_wina_scores_rank_by_norm_and_magnitude(oracle_lib):
+    # equal norms give the |x| tiers; equal |x| gives the tiers of the norms (column order on ties)
+    rng = np.random.default_rng(22)
+    x = synth.laplace((500,), 2, 5).numpy()
+    ones = np.full(500, 4.0, np.float32)  # a power of two: the products keep the order exactly
+    kf, ka = 120, 150
+    _, t_x, *_ = oracle_lib.tiers(x, oracle_lib.MODE_TOPK, k_full=kf, k_approx=ka)
+    _, t_s, *_ = oracle_lib.tiers(oracle_lib.wina_scores(x, ones), oracle_lib.MODE_TOPK,
+                                  k_full=kf, k_approx=ka)
+    assert np.array_equal(t_x, t_s)
+    norms = rng.uniform(0.1, 2.0, 500).astype(np.float32)
+    _, t_n, *_ = oracle_lib.tiers(oracle_lib.wina_scores(np.full(500, -0.5, np.float32), norms),
+                                  oracle_lib.MODE_TOPK, k_full=kf, k_approx=ka)
+    rank = np.argsort(-norms, kind="stable")
+    want = np.zeros(500, np.uint8)
+    want[rank[:kf]] = 2
+    want[rank[kf:kf + ka]] = 1
+    assert np.array_equal(t_n, want)
+    # the score is the fp32 product itself
+    s = oracle_lib.wina_scores(np.array([-3.0, 0.1], np.float32), np.array([0.5, 3.0], np.float32))
+    assert s[0] == np.float32(1.5) and s[1] == np.float32(0.1) * np.float32(3.0)

@@ -216,7 +216,8 @@ spax_status spax_tiered_gemv(const spax_packed* W, const float* x, const int32_t
 }
 
 static spax_status masked_gemv_common(const spax_packed* W, const float* x, bool swiglu,
-                                      float* x_out, const spax_mask_params* p, float* y,
+                                      float* x_out, const float* norms,
+                                      const spax_mask_params* p, float* y,
                                       uint8_t* tier, int32_t* full_idx, int32_t* approx_idx,
                                       int32_t* counts, int32_t* status, void* ws, size_t ws_bytes,
                                       void* stream) {
@@ -249,16 +250,31 @@ static spax_status masked_gemv_common(const spax_packed* W, const float* x, bool
   a.d_in = W->d_in;
   a.full_fmt = W->full_fmt;
   a.dense = false;
-  return launch_status(launch_masked_gemv(a, q, swiglu, x_out, tier, full_idx, approx_idx, counts,
-                                          pl, static_cast<cudaStream_t>(stream)));
+  return launch_status(launch_masked_gemv(a, q, swiglu, x_out, norms, tier, full_idx, approx_idx,
+                                          counts, pl, static_cast<cudaStream_t>(stream)));
 }
 
 spax_status spax_masked_gemv(const spax_packed* W, const float* x, const spax_mask_params* p,
                              float* y, uint8_t* tier, int32_t* full_idx, int32_t* approx_idx,
                              int32_t* counts, int32_t* status, void* ws, size_t ws_bytes,
                              void* stream) {
-  return masked_gemv_common(W, x, false, nullptr, p, y, tier, full_idx, approx_idx, counts, status,
-                            ws, ws_bytes, stream);
+  return masked_gemv_common(W, x, false, nullptr, nullptr, p, y, tier, full_idx, approx_idx, counts,
+                            status, ws, ws_bytes, stream);
+}
+
+spax_status spax_masked_gemv_wina(const spax_packed* W, const float* x, const float* norms,
+                                  const spax_mask_params* p, float* y, uint8_t* tier,
+                                  int32_t* full_idx, int32_t* approx_idx, int32_t* counts,
+                                  int32_t* status, void* ws, size_t ws_bytes, void* stream) {
+  if (!norms) return SPAX_ERR_ARG;
+  return masked_gemv_common(W, x, false, nullptr, norms, p, y, tier, full_idx, approx_idx, counts,
+                            status, ws, ws_bytes, stream);
+}
+
+spax_status spax_column_norms(const void* W, int d_out, int d_in, float* norms, void* stream) {
+  if (!W || !norms) return SPAX_ERR_ARG;
+  if (d_out < 1 || d_in < 1) return SPAX_ERR_SHAPE;
+  return launch_status(launch_column_norms(W, d_out, d_in, norms, static_cast<cudaStream_t>(stream)));
 }
 
 spax_status spax_masked_gemv_swiglu(const spax_packed* W, const float* gu,
@@ -266,8 +282,8 @@ spax_status spax_masked_gemv_swiglu(const spax_packed* W, const float* gu,
                                     uint8_t* tier, int32_t* full_idx, int32_t* approx_idx,
                                     int32_t* counts, int32_t* status, void* ws, size_t ws_bytes,
                                     void* stream) {
-  return masked_gemv_common(W, gu, true, x_out, p, y, tier, full_idx, approx_idx, counts, status,
-                            ws, ws_bytes, stream);
+  return masked_gemv_common(W, gu, true, x_out, nullptr, p, y, tier, full_idx, approx_idx, counts,
+                            status, ws, ws_bytes, stream);
 }
 
 spax_status spax_dense_gemv(const void* Wt, const float* x, float* y, int d_out, int d_in,

@@ -84,6 +84,7 @@ struct GemvParams {
   int list_bytes;  // 0 for the list-driven kernels
   int swiglu;      // fused only: x holds [g; u] and x_j = swiglu_x(g_j, u_j)
   float* x_out;    // fused swiglu only: the token's x (lead CTA; may be null)
+  const float* norms;  // fused only, may be null: rank by the WINA score |x_j| * norms[j]
 };
 
 // Code -> float: (word & (mask << p)) | bits(C) is the float C + code, exactly, when C = 2^(23-p)
@@ -182,6 +183,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
     pdl_launch_dependents();
     if (p.swiglu)
       select_fetch_swiglu(p.x, p.d_in, keys, tile == 0 && split == 0 ? p.x_out : nullptr);
+    else if (p.norms)
+      select_fetch_scored(p.x, p.norms, p.d_in, keys);
     else
       select_fetch(p.x, p.d_in, keys);
     const uint32_t ts = __float_as_uint(p.prm.t_skip) & 0x7FFFFFFFu;
@@ -225,8 +228,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
       }
       // signed x of this split's first kGemvMeta positions of each list, kept in the metadata
       // arrays (idle in this kernel) for the product: no reload, no recomputation
-      const int nfl = min(kGemvMeta, Kf > split ? (Kf - split + S - 1) / S : 0);
-      const int nal = min(kGemvMeta, Ka > split ? (Ka - split + S - 1) / S : 0);
+      // (not with the WINA score: its keys are scores, so the product reads x itself)
+      const int nfl = p.norms ? 0 : min(kGemvMeta, Kf > split ? (Kf - split + S - 1) / S : 0);
+      const int nal = p.norms ? 0 : min(kGemvMeta, Ka > split ? (Ka - split + S - 1) / S : 0);
       for (int i = tid; i < nfl; i += kGemvThreads)
         reinterpret_cast<float*>(meta_col_f)[i] = select_signed_x(keys, sgn, list[split + S * i]);
       for (int i = tid; i < nal; i += kGemvThreads)
@@ -288,15 +292,16 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
 
   // x of local position i of this split's approximate / full list: the fused kernel's stash
   // (first kGemvMeta positions), else x of the column
+  const int xs_lim = (FUSED && !p.norms) ? kGemvMeta : 0;  // positions the stash holds
   auto xA = [&](int i, int col) -> float {
     if constexpr (FUSED) {
-      if (i < kGemvMeta) return reinterpret_cast<const float*>(meta_col_a)[i];
+      if (i < xs_lim) return reinterpret_cast<const float*>(meta_col_a)[i];
     }
     return xval(col);
   };
   auto xF = [&](int i, int col) -> float {
     if constexpr (FUSED) {
-      if (i < kGemvMeta) return reinterpret_cast<const float*>(meta_col_f)[i];
+      if (i < xs_lim) return reinterpret_cast<const float*>(meta_col_f)[i];
     }
     return xval(col);
   };
@@ -767,13 +772,14 @@ cudaError_t launch_gemv(const GemvLaunch& a, const GemvPlan& pl, cudaStream_t st
 }
 
 cudaError_t launch_masked_gemv(const GemvLaunch& a, const spax_mask_params& prm, bool swiglu,
-                               float* x_out, uint8_t* tier, int32_t* full_idx,
+                               float* x_out, const float* norms, uint8_t* tier, int32_t* full_idx,
                                int32_t* approx_idx, int32_t* counts, const GemvPlan& pl,
                                cudaStream_t stream) {
   GemvParams gp = make_params(a, pl);
   gp.prm = prm;
   gp.swiglu = swiglu ? 1 : 0;
   gp.x_out = swiglu ? x_out : nullptr;
+  gp.norms = swiglu ? nullptr : norms;
   gp.tier_out = tier;
   gp.fidx_out = full_idx;
   gp.aidx_out = approx_idx;

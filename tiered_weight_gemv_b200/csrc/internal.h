@@ -37,8 +37,9 @@ cudaError_t launch_gemv(const GemvLaunch& a, const GemvPlan& plan, cudaStream_t 
 // The mask and the GEMV in one launch (every CTA computes the token's lists itself); the tier,
 // list and count outputs may be null. Shared memory it needs for a plan and d_in.
 // swiglu: a.x holds [g; u] (2 * d_in) and x_j = silu(g_j) * u_j (written to x_out when set).
+// norms (may be null): rank columns by the WINA score |x_j| * norms[j] instead of |x_j|.
 cudaError_t launch_masked_gemv(const GemvLaunch& a, const spax_mask_params& prm, bool swiglu,
-                               float* x_out, uint8_t* tier, int32_t* full_idx,
+                               float* x_out, const float* norms, uint8_t* tier, int32_t* full_idx,
                                int32_t* approx_idx, int32_t* counts, const GemvPlan& plan,
                                cudaStream_t stream);
 size_t masked_gemv_smem_bytes(const GemvPlan& plan, int d_in);
@@ -49,6 +50,8 @@ cudaError_t launch_mask(const float* x, int d_in, const spax_mask_params& p, uin
 
 cudaError_t launch_pack(const void* W, int d_out, int d_in, int full_fmt, void* full, void* approx,
                         cudaStream_t stream);
+cudaError_t launch_column_norms(const void* W, int d_out, int d_in, float* norms,
+                                cudaStream_t stream);
 
 size_t calibrate_ws_bytes();
 cudaError_t launch_calibrate(const float* X, long long M, long long idx_skip, long long idx_full,

@@ -130,6 +130,44 @@ __global__ void __launch_bounds__(256) pack_kernel(const uint16_t* __restrict__ 
   }
 }
 
+// Column norms for the WINA score (TopK-Guided §C.1): one thread per column sums the squares of
+// its d_out bf16 values in fp64, in row order (a fixed order: every square is exact in fp64, the
+// sum rounds the same way wherever this definition is followed), then a correctly rounded sqrt
+// and one rounding to fp32. The loads of eight rows are issued together; a warp reads 32
+// neighbouring columns of a row (64 contiguous bytes).
+__global__ void __launch_bounds__(256) column_norm_kernel(const uint16_t* __restrict__ W,
+                                                         int d_out, int d_in,
+                                                         float* __restrict__ norms) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= d_in) return;
+  const uint16_t* col = W + j;
+  double acc = 0.0;
+  int r = 0;
+  for (; r + 8 <= d_out; r += 8) {
+    uint16_t v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = __ldg(col + (size_t)(r + k) * d_in);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const double w = (double)__uint_as_float((uint32_t)v[k] << 16);
+      acc = __dadd_rn(acc, __dmul_rn(w, w));
+    }
+  }
+  for (; r < d_out; ++r) {
+    const double w = (double)__uint_as_float((uint32_t)__ldg(col + (size_t)r * d_in) << 16);
+    acc = __dadd_rn(acc, __dmul_rn(w, w));
+  }
+  norms[j] = __double2float_rn(__dsqrt_rn(acc));
+}
+
+cudaError_t launch_column_norms(const void* W, int d_out, int d_in, float* norms,
+                                cudaStream_t stream) {
+  return launch_pdl(column_norm_kernel, dim3((d_in + 255) / 256), dim3(256), 0, stream,
+                    static_cast<const uint16_t*>(W), d_out, d_in, norms);
+}
+
 cudaError_t launch_pack(const void* W, int d_out, int d_in, int full_fmt, void* full, void* approx,
                         cudaStream_t stream) {
   const int nrec2_groups = ((d_out + 511) / 512) * 4;

@@ -160,6 +160,45 @@ __device__ __forceinline__ void select_fetch_swiglu(const float* __restrict__ gu
   __syncthreads();
 }
 
+// WINA score keys: keys[j] = bits(|x_j| * norm_j) (one correctly rounded fp32 product; x and
+// the norms read in batches ahead of the arithmetic), the tail of the last quad zero. Ends with
+// a barrier.
+__device__ __forceinline__ void select_fetch_scored(const float* __restrict__ x,
+                                                    const float* __restrict__ norms, int d,
+                                                    uint32_t* __restrict__ keys) {
+  const int tid = threadIdx.x;
+  const int nfull = d >> 2;
+  auto score = [](float a, float n) { return __float_as_uint(__fmul_rn(fabsf(a), n)); };
+  if (((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(norms)) & 15u) == 0) {
+    constexpr int kB = 6;
+    for (int q0 = tid; q0 < nfull; q0 += kB * kSelThreads) {
+      float4 a[kB], n[kB];
+#pragma unroll
+      for (int k = 0; k < kB; ++k) {
+        const int q = q0 + k * kSelThreads;
+        if (q < nfull) {
+          a[k] = __ldg(reinterpret_cast<const float4*>(x) + q);
+          n[k] = __ldg(reinterpret_cast<const float4*>(norms) + q);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < kB; ++k) {
+        const int q = q0 + k * kSelThreads;
+        if (q < nfull)
+          reinterpret_cast<uint4*>(keys)[q] = make_uint4(score(a[k].x, n[k].x), score(a[k].y, n[k].y),
+                                                         score(a[k].z, n[k].z), score(a[k].w, n[k].w));
+      }
+    }
+  } else {
+    for (int j = tid; j < 4 * nfull; j += kSelThreads) keys[j] = score(__ldg(x + j), __ldg(norms + j));
+  }
+  if (tid < 4 && (d & 3)) {
+    const int j = 4 * nfull + tid;
+    keys[j] = j < d ? score(__ldg(x + j), __ldg(norms + j)) : 0u;
+  }
+  __syncthreads();
+}
+
 // Sign bits of quad q's four x values (bit e for x[4q + e]), for select_signed_x.
 __device__ __forceinline__ uint8_t quad_signs(uint4 v) {
   return (uint8_t)((v.x >> 31) | ((v.y >> 31) << 1) | ((v.z >> 31) << 2) | ((v.w >> 31) << 3));

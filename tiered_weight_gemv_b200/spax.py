@@ -60,6 +60,10 @@ _SIGS = {
     "spax_dense_gemv": ([_P, _P, _P, _I, _I, _P, _P, _Z, _P], _I),
     "spax_masked_gemv": ([ctypes.POINTER(spax_packed), _P, ctypes.POINTER(spax_mask_params), _P,
                           _P, _P, _P, _P, _P, _P, _Z, _P], _I),
+    "spax_masked_gemv_wina": ([ctypes.POINTER(spax_packed), _P, _P,
+                               ctypes.POINTER(spax_mask_params), _P, _P, _P, _P, _P, _P, _P, _Z,
+                               _P], _I),
+    "spax_column_norms": ([_P, _I, _I, _P, _P], _I),
     "spax_masked_gemv_swiglu": ([ctypes.POINTER(spax_packed), _P, ctypes.POINTER(spax_mask_params),
                                  _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P], _I),
     "spax_tiered_gemv_fixed_scratch": ([ctypes.POINTER(spax_packed), _P, _P, _P, _P, _P, _P, _P],
@@ -255,6 +259,35 @@ def spax_masked_gemv(W: PackedMatrix, x: torch.Tensor, params: spax_mask_params,
     _check("spax_masked_gemv", _lib.spax_masked_gemv(
         ctypes.byref(d), _dev(x, torch.float32, "x"), ctypes.byref(params),
         _dev(y, torch.float32, "y"), _dev(tier, torch.uint8, "tier"),
+        _dev(full_idx, torch.int32, "full_idx"), _dev(approx_idx, torch.int32, "approx_idx"),
+        _dev(counts, torch.int32, "counts"), _dev(status, torch.int32, "status"),
+        _dev(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def spax_column_norms(W: torch.Tensor, norms: torch.Tensor, stream=None) -> None:
+    """Per-column Euclidean norms of the row-major bf16 W (for the WINA score)."""
+    d_out, d_in = W.shape
+    if norms.numel() < d_in:
+        raise ValueError("norms too small")
+    _check("spax_column_norms", _lib.spax_column_norms(
+        _dev(W, torch.bfloat16, "W"), d_out, d_in, _dev(norms, torch.float32, "norms"),
+        _stream(stream)))
+
+
+def spax_masked_gemv_wina(W: PackedMatrix, x: torch.Tensor, norms: torch.Tensor,
+                          params: spax_mask_params, y: torch.Tensor, status: torch.Tensor,
+                          ws: torch.Tensor, tier=None, full_idx=None, approx_idx=None, counts=None,
+                          stream=None, desc=None) -> None:
+    """spax_masked_gemv ranking columns by the WINA score |x_j| * norms[j]."""
+    if x.numel() != W.d_in or norms.numel() != W.d_in or y.numel() != W.d_out:
+        raise ValueError("x / norms / y sizes do not match W")
+    for t, n in ((tier, W.d_in), (full_idx, W.d_in), (approx_idx, W.d_in), (counts, 4)):
+        if t is not None and t.numel() < n:
+            raise ValueError("mask output too small")
+    d = W.desc() if desc is None else desc
+    _check("spax_masked_gemv_wina", _lib.spax_masked_gemv_wina(
+        ctypes.byref(d), _dev(x, torch.float32, "x"), _dev(norms, torch.float32, "norms"),
+        ctypes.byref(params), _dev(y, torch.float32, "y"), _dev(tier, torch.uint8, "tier"),
         _dev(full_idx, torch.int32, "full_idx"), _dev(approx_idx, torch.int32, "approx_idx"),
         _dev(counts, torch.int32, "counts"), _dev(status, torch.int32, "status"),
         _dev(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream)))
