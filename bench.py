@@ -560,7 +560,96 @@ def run_extras(args, dev):
     }
     del layer
     torch.cuda.empty_cache()
+    out["host_link_offload"] = run_host_link(args, dev)
+    torch.cuda.empty_cache()
     return out
+
+
+def run_host_link(args, dev):
+    """The pages' own setting: the Llama-2-7B block's packed pools in page-locked host memory, read
+    by the same kernels over the host link (zero-copy), masked GEMV against dense. The roofline is
+    a measured host-to-device copy of pinned memory; the bytes that must cross the link are the
+    selected weights (x, lists and y stay in device memory)."""
+    from tiered_weight_gemv_b200 import spax
+
+    n_tok, n_rep = 8, 2
+    steps, warmup = max(3, min(args.steps, 5)), args.warmup
+    stream = torch.cuda.Stream(device=dev)
+    mats = make_weights(dev)
+    xs = make_inputs(mats, n_tok, dev)
+    sites = {}
+    for name, d_out, d_in, _ in SITES:
+        pm = spax.alloc_packed(d_out, d_in, spax.FULL_BF16, device=dev)
+        spax.spax_pack_weights(mats[name], spax.FULL_BF16, pm)
+        torch.cuda.synchronize()
+        reps = [spax.packed_to_host(pm) for _ in range(n_rep)]
+        del pm
+        kf, ka = k_counts(d_in)
+        sites[name] = dict(reps=reps, descs=[r.desc() for r in reps], d_out=d_out, d_in=d_in, kf=kf,
+                           ka=ka, prm=spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka),
+                           y=torch.empty(n_tok, d_out, device=dev),
+                           st=torch.zeros(1, dtype=torch.int32, device=dev),
+                           ws=spax.alloc_workspace(spax.OP_TIERED_GEMV, d_out, d_in, device=dev),
+                           dws=spax.alloc_workspace(spax.OP_DENSE_GEMV, d_out, d_in, device=dev))
+    del mats
+    torch.cuda.synchronize()
+
+    def masked():
+        for t in range(n_tok):
+            for name, *_ in SITES:
+                b = sites[name]
+                r = t % n_rep
+                spax.spax_masked_gemv(b["reps"][r], xs[name][t], b["prm"], b["y"][t], b["st"], b["ws"],
+                                      desc=b["descs"][r])
+
+    def dense():
+        for t in range(n_tok):
+            for name, *_ in SITES:
+                b = sites[name]
+                spax.spax_dense_gemv(b["reps"][t % n_rep].full, xs[name][t], b["y"][t], b["d_out"],
+                                     b["d_in"], b["st"], b["dws"])
+
+    res = {}
+    for label, fn in (("masked", masked), ("dense", dense)):
+        with torch.cuda.stream(stream):
+            fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        res[label] = time_graph(g, steps, warmup, stream) * 1000 / n_tok  # us per token-layer
+        del g
+    for name, *_ in SITES:
+        if int(sites[name]["st"].item()) != 0:
+            raise RuntimeError(f"device status {int(sites[name]['st'].item())} (host pools, {name})")
+    # the link's measured rate: one 1 GiB copy of pinned host memory to the device
+    src = torch.empty(1 << 30, dtype=torch.uint8, pin_memory=True)
+    dst = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            dst.copy_(src, non_blocking=True)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(3):
+            dst.copy_(src, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    copy_gbps = 3 * (1 << 30) / (e0.elapsed_time(e1) * 1e-3) / 1e9
+    link_bytes = sum(spax.spax_weight_bytes(b["d_out"], spax.FULL_BF16, b["kf"], b["ka"])
+                     for b in sites.values())
+    dense_bytes = sum(2 * b["d_out"] * b["d_in"] for b in sites.values())
+    achieved = link_bytes / (res["masked"] * 1e-6) / 1e9
+    return {"tokens": n_tok, "replicas_in_host_memory": n_rep,
+            "masked_us_per_token_layer": round(res["masked"], 1),
+            "dense_us_per_token_layer": round(res["dense"], 1),
+            "speedup_vs_dense": round(res["dense"] / res["masked"], 3),
+            "selected_bytes_per_token_layer": link_bytes,
+            "dense_bytes_per_token_layer": dense_bytes,
+            "masked_link_GBps": round(achieved, 1),
+            "dense_link_GBps": round(dense_bytes / (res["dense"] * 1e-6) / 1e9, 1),
+            "h2d_copy_GBps": round(copy_gbps, 1),
+            "masked_frac_of_copy": round(achieved / copy_gbps, 4)}
 
 
 def fit_c0_bw(points):
@@ -707,6 +796,9 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=24)
     ap.add_argument("--ref-tokens", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--host-link-only", action="store_true",
+                    help="profiling aid: run only the host-link offload measurement (pools in "
+                         "page-locked host memory) and print its JSON; not the benchmark line")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the measurements beside the headline (dequant vs load, the "
                          "Llama-3-8B sweep and fit, dense and torch.mv)")
@@ -719,6 +811,12 @@ def main():
     try:
         if args.impl == "reference":
             return run_reference(args, rank, world)
+        if args.host_link_only:
+            torch.cuda.set_device(local)
+            if rank == 0:
+                print(json.dumps({"host_link_offload": run_host_link(args, torch.device("cuda", local))}),
+                      flush=True)
+            return 0
         res, sites, tot_bytes, tot_ms, lps, h2d, d2h, clocks, host = run_gpu(args, rank, world, local)
         ms = res["fused"]
         value = us_per_token_layer(ms, args.tokens, world)

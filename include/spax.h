@@ -104,7 +104,14 @@ typedef struct {
   int32_t delta_bp;
 } spax_mask_params;
 
-/* A packed matrix: both pools in device memory, owned by the caller. */
+/*
+ * A packed matrix: both pools owned by the caller, in device memory or in page-locked host
+ * memory mapped into the device address space (unified addressing: the host pointer of a
+ * cudaHostAlloc / cudaHostRegister allocation). With host pools the GEMV kernels read the
+ * selected column segments straight over the host link, which is the offloaded-weights setting
+ * of the SpAx Abstract and of the eigenradar commentary ("The route outside GPU memory"): only
+ * the full and approximate tiers' bytes cross the link. Results are identical to device pools.
+ */
 typedef struct {
   int32_t d_out;
   int32_t d_in;

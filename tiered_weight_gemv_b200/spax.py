@@ -106,6 +106,13 @@ def _dev(t, dtype=None, name="tensor"):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _dev_or_pinned(t, name="tensor"):
+    """A weight pool: device memory, or page-locked host memory (mapped into the device)."""
+    if isinstance(t, torch.Tensor) and not t.is_cuda and t.is_pinned() and t.is_contiguous():
+        return ctypes.c_void_p(t.data_ptr())
+    return _dev(t, None, name)
+
+
 def _stream(stream):
     s = torch.cuda.current_stream() if stream is None else stream
     return ctypes.c_void_p(s.cuda_stream)
@@ -189,6 +196,17 @@ def alloc_packed(d_out: int, d_in: int, full_fmt: int, device="cuda") -> PackedM
     return PackedMatrix(d_out, d_in, full_fmt,
                         torch.empty(fb, dtype=torch.uint8, device=device),
                         torch.empty(ab, dtype=torch.uint8, device=device))
+
+
+def packed_to_host(pm: PackedMatrix) -> PackedMatrix:
+    """A copy of a packed matrix in page-locked host memory. Unified addressing maps such memory
+    into the device address space, so the GEMV kernels read the pools straight over the host
+    link (the offloaded-weights setting); the descriptor's pointers are the host pointers."""
+    full = torch.empty(pm.full.numel(), dtype=torch.uint8, pin_memory=True)
+    approx = torch.empty(pm.approx.numel(), dtype=torch.uint8, pin_memory=True)
+    full.copy_(pm.full)
+    approx.copy_(pm.approx)
+    return PackedMatrix(pm.d_out, pm.d_in, pm.full_fmt, full, approx)
 
 
 def spax_pack_weights(W: torch.Tensor, full_fmt: int, dst: PackedMatrix, stream=None) -> None:
@@ -337,7 +355,7 @@ def spax_dense_gemv(Wt: torch.Tensor, x: torch.Tensor, y: torch.Tensor, d_out: i
     if x.numel() != d_in or y.numel() != d_out or Wt.numel() * Wt.element_size() < 2 * d_in * d_out:
         raise ValueError("sizes do not match")
     _check("spax_dense_gemv", _lib.spax_dense_gemv(
-        _dev(Wt, None, "Wt"), _dev(x, torch.float32, "x"), _dev(y, torch.float32, "y"), d_out,
+        _dev_or_pinned(Wt, "Wt"), _dev(x, torch.float32, "x"), _dev(y, torch.float32, "y"), d_out,
         d_in, _dev(status, torch.int32, "status"), _dev(ws, None, "ws"),
         ws.numel() * ws.element_size(), _stream(stream)))
 
