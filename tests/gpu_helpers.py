@@ -79,8 +79,30 @@ def oracle_params(params) -> dict:
                 s_below_full_bp=params.s_below_full_bp, delta_bp=params.delta_bp)
 
 
-def check_token(gm: GpuMatrix, pools, x: torch.Tensor, params, rows=None):
-    """Run one token on both sides and compare; pools = the oracle's own (full, approx) pools."""
+def check_masked_equals_two_call(gm: GpuMatrix, x: torch.Tensor, params, g: dict):
+    """spax_masked_gemv (mask + GEMV in one launch) on the same token: its tiers, lists, counts
+    and y must equal the two-call results g bit for bit (same rule, same product order)."""
+    d_in = gm.d_in
+    tier = torch.full((d_in,), 7, dtype=torch.uint8, device=x.device)
+    fidx = torch.full((d_in,), -5, dtype=torch.int32, device=x.device)
+    aidx = torch.full((d_in,), -5, dtype=torch.int32, device=x.device)
+    counts = torch.full((4,), -5, dtype=torch.int32, device=x.device)
+    y = torch.full((gm.d_out,), float("nan"), device=x.device)
+    st = torch.zeros(1, dtype=torch.int32, device=x.device)
+    spax.spax_masked_gemv(gm.pm, x, params, y, st, gm.ws, tier=tier, full_idx=fidx,
+                          approx_idx=aidx, counts=counts)
+    torch.cuda.synchronize()
+    c = counts.cpu().numpy()
+    assert st.item() == 0 and np.array_equal(c, g["counts"])
+    assert np.array_equal(tier.cpu().numpy(), g["tier"])
+    assert np.array_equal(fidx[: c[0]].cpu().numpy(), g["fidx"])
+    assert np.array_equal(aidx[: c[1]].cpu().numpy(), g["aidx"])
+    assert np.array_equal(y.cpu().numpy(), g["y"]), "masked GEMV y differs from the two-call y"
+
+
+def check_token(gm: GpuMatrix, pools, x: torch.Tensor, params, rows=None, masked=True):
+    """Run one token on both sides and compare; pools = the oracle's own (full, approx) pools.
+    masked: also run the one-launch masked GEMV and require the two-call results bit for bit."""
     g = gm.token(x, params)
     xn = x.cpu().numpy()
     op = oracle_params(params)
@@ -92,4 +114,7 @@ def check_token(gm: GpuMatrix, pools, x: torch.Tensor, params, rows=None):
     full_o, approx_o = pools
     y_ref = oracle.tiered_gemv(full_o, approx_o, gm.fmt, gm.d_out, gm.d_in, xn, tier, rows=rows)
     y = g["y"] if rows is None else g["y"][rows]
-    return check_y(y, y_ref), g
+    rel = check_y(y, y_ref)
+    if masked and gm.d_in <= spax.MASK_MAX_DIN:
+        check_masked_equals_two_call(gm, x, params, g)
+    return rel, g
