@@ -51,16 +51,14 @@ constexpr int kStage2Bytes = 16 * 144;      // one batch of 2-bit records
 constexpr int kStageRecBytes = 2 * kStage2Bytes;  // two 2-bit batches (>= one int4 batch, 16 * 272)
 constexpr int kStageWarpBytes = kStageRecBytes + 16 * 16;  // + 4 coefficients per column
 
-template <int RG>
-struct GemvCfg {
-  static constexpr int R = 512 * RG;          // rows per tile
-  static constexpr int CG = kGemvWarps / RG;  // column groups
-  static constexpr int kSlotFloats = (R / 32) * 36;  // combine slot: 36 floats per 32 rows
-  static constexpr size_t kSmemBytes = size_t(2) * kGemvMeta * 4 + size_t(CG) * kSlotFloats * 4 +
-                                       size_t(kGemvWarps) * kStageWarpBytes;
-  static_assert(CG >= 4, "reduction scratch must fit the combine area");
-  static_assert(kBatch4 * 272 <= kStageRecBytes && 2 * kBatch2 * 144 <= kStageRecBytes, "staging");
-};
+// Row tile of R = 512 RG rows (RG = 1, 2 or 4, a launch parameter): warp (rg, cg) takes rows
+// [512 rg, 512 rg + 512) of the tile and every CG-th column of the CTA's share, CG = 16 / RG.
+// One kernel image serves every tile height, so the launches of a decoder layer (whose shapes
+// want different tiles) all run the same code and keep it warm in the instruction caches.
+constexpr int kCombineFloats = kGemvWarps * 576;  // CG slots of (R / 32) * 36 floats, any RG
+constexpr size_t kGemvSmemBytes = size_t(2) * kGemvMeta * 4 + size_t(kCombineFloats) * 4 +
+                                  size_t(kGemvWarps) * kStageWarpBytes;
+static_assert(kBatch4 * 272 <= kStageRecBytes && 2 * kBatch2 * 144 <= kStageRecBytes, "staging");
 
 struct GemvParams {
   const uint8_t* full;
@@ -82,6 +80,7 @@ struct GemvParams {
   int32_t* aidx_out;
   int32_t* counts_out;
   int list_bytes;  // 0 for the list-driven kernels
+  int RG;          // row tile R = 512 * RG (1, 2 or 4)
   int swiglu;      // fused only: x holds [g; u] and x_j = swiglu_x(g_j, u_j)
   float* x_out;    // fused swiglu only: the token's x (lead CTA; may be null)
   const float* norms;  // fused only, may be null: rank by the WINA score |x_j| * norms[j]
@@ -139,10 +138,14 @@ __host__ __device__ inline size_t fused_select_bytes(int d) {
 
 // FUSED: the kernel first runs the tier rule on x itself (select.cuh: every CTA computes the
 // same lists, staged in its shared memory), then reads its split's positions from there.
-template <int RG, int FMT, bool DENSE, bool FUSED>
+// RGT: the row-tile factor fixed at compile time (1, 2, 4), or 0 for the launch's p.RG. The tiered
+// kernels take 0 (one image for every shape of a layer); the dense baseline, a pure stream that
+// gains from the constant, keeps one image per tile height.
+template <int RGT, int FMT, bool DENSE, bool FUSED>
 __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const GemvParams p) {
-  using C = GemvCfg<RG>;
-  constexpr int R = C::R, CG = C::CG, U = kGemvU;
+  constexpr int U = kGemvU;
+  const int RG = RGT > 0 ? RGT : p.RG, R = 512 * RG, CG = kGemvWarps / RG;
+  const int kSlotFloats = RG * 576;  // combine slot of a column group: 36 floats per 32 rows
   static_assert(FMT == SPAX_FULL_BF16 || !DENSE, "the dense GEMV reads the bf16 pool");
   static_assert(!(DENSE && FUSED), "the dense GEMV has no mask");
   extern __shared__ __align__(128) uint8_t smem[];
@@ -163,7 +166,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
   const bool v0 = rb + 8 * lane < p.d_out;   // lane's first 8-row chunk is inside the matrix
   const bool v1 = rb + 256 + 8 * lane < p.d_out;
   // per-warp staging buffer: kBatch records, then their coefficients x*scale per 128-row group
-  uint8_t* stage = reinterpret_cast<uint8_t*>(red + CG * C::kSlotFloats) + warp * kStageWarpBytes;
+  uint8_t* stage = reinterpret_cast<uint8_t*>(red + kCombineFloats) + warp * kStageWarpBytes;
   const uint32_t stage_s = smem_u32(stage);
   const uint32_t coef_s = stage_s + kStageRecBytes;
 
@@ -586,7 +589,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
   if (wrows) {
     // remove the mantissa constants: 2-bit rows 4i+{0,1,2,3} carry {256,64,16,4}*Σc, int4 even
     // rows (256+8)*Σc and odd rows (16+8)*Σc; add Σ x*min for the 2-bit tier
-    float* slot = red + cg * C::kSlotFloats;
+    float* slot = red + cg * kSlotFloats;
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
       const float sa = b ? sumA1 : sumA0, ba = b ? baseA1 : baseA0, s4 = b ? sum41 : sum40;
@@ -610,9 +613,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
   // rows 4i..4i+3 of the tile: the column groups' slots summed in group order
   auto combined_rows = [&](int i) -> float4 {
     float4 v = reinterpret_cast<const float4*>(red + red_row(4 * i))[0];
-#pragma unroll
+#pragma unroll 3
     for (int c = 1; c < CG; ++c) {
-      const float4 w = reinterpret_cast<const float4*>(red + c * C::kSlotFloats + red_row(4 * i))[0];
+      const float4 w = reinterpret_cast<const float4*>(red + c * kSlotFloats + red_row(4 * i))[0];
       v.x += w.x;
       v.y += w.y;
       v.z += w.z;
@@ -712,10 +715,10 @@ bool make_gemv_plan(int d_out, int d_in, int full_fmt, int sm_count, GemvPlan* p
   return true;
 }
 
-template <int RG, int FMT, bool DENSE, bool FUSED>
+template <int RGT, int FMT, bool DENSE, bool FUSED>
 static cudaError_t launch_one(const GemvParams& gp, const GemvPlan& pl, size_t smem,
                               cudaStream_t stream) {
-  auto kern = tiered_gemv_kernel<RG, FMT, DENSE, FUSED>;
+  auto kern = tiered_gemv_kernel<RGT, FMT, DENSE, FUSED>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), (int)smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(pl.T, pl.S), dim3(kGemvThreads), smem, stream, gp);
@@ -724,19 +727,20 @@ static cudaError_t launch_one(const GemvParams& gp, const GemvPlan& pl, size_t s
 template <int FMT, bool DENSE, bool FUSED>
 static cudaError_t launch_r(const GemvParams& gp, const GemvPlan& pl, size_t smem,
                             cudaStream_t stream) {
-  if (pl.R == 512) return launch_one<1, FMT, DENSE, FUSED>(gp, pl, smem, stream);
-  if (pl.R == 1024) return launch_one<2, FMT, DENSE, FUSED>(gp, pl, smem, stream);
-  return launch_one<4, FMT, DENSE, FUSED>(gp, pl, smem, stream);
+  if constexpr (DENSE) {
+    if (pl.R == 512) return launch_one<1, FMT, DENSE, FUSED>(gp, pl, smem, stream);
+    if (pl.R == 1024) return launch_one<2, FMT, DENSE, FUSED>(gp, pl, smem, stream);
+    return launch_one<4, FMT, DENSE, FUSED>(gp, pl, smem, stream);
+  } else {
+    return launch_one<0, FMT, DENSE, FUSED>(gp, pl, smem, stream);
+  }
 }
 
-static size_t gemv_smem_bytes(int R) {
-  return R == 512 ? GemvCfg<1>::kSmemBytes
-                  : (R == 1024 ? GemvCfg<2>::kSmemBytes : GemvCfg<4>::kSmemBytes);
-}
+static size_t gemv_smem_bytes() { return kGemvSmemBytes; }
 
-size_t masked_gemv_smem_bytes(const GemvPlan& pl, int d_in) {
+size_t masked_gemv_smem_bytes(const GemvPlan& /*pl: every tile height takes the same*/, int d_in) {
   const size_t meta = size_t(2) * kGemvMeta * 4;
-  const size_t gemv = gemv_smem_bytes(pl.R) - meta;  // combine + staging areas
+  const size_t gemv = gemv_smem_bytes() - meta;  // combine + staging areas
   const size_t sel = fused_select_bytes(d_in);
   return meta + select_list_bytes(d_in) + (gemv > sel ? gemv : sel);
 }
@@ -759,13 +763,14 @@ static GemvParams make_params(const GemvLaunch& a, const GemvPlan& pl) {
   gp.d_out = a.d_out;
   gp.d_in = a.d_in;
   gp.S = pl.S;
+  gp.RG = pl.R / 512;
   gp.list_bytes = 0;
   return gp;
 }
 
 cudaError_t launch_gemv(const GemvLaunch& a, const GemvPlan& pl, cudaStream_t stream) {
   const GemvParams gp = make_params(a, pl);
-  const size_t smem = gemv_smem_bytes(pl.R);
+  const size_t smem = gemv_smem_bytes();
   if (a.dense) return launch_r<SPAX_FULL_BF16, true, false>(gp, pl, smem, stream);
   if (a.full_fmt == SPAX_FULL_BF16) return launch_r<SPAX_FULL_BF16, false, false>(gp, pl, smem, stream);
   return launch_r<SPAX_FULL_INT4_G128, false, false>(gp, pl, smem, stream);
