@@ -109,7 +109,9 @@ __device__ __forceinline__ void select_fetch(const float* __restrict__ x, int d,
 
 // x_j = swiglu_x(g_j, u_j) from gu = [g; u] (2 d values) -> keys[] as raw fp32 bits, the tail
 // of the last quad zero; x_out (may be null) receives x. Ends with a barrier.
-__device__ __forceinline__ void select_fetch_swiglu(const float* __restrict__ gu, int d,
+// Out of line (as is select_fetch_scored): only the chained-layer entry point runs it, and code
+// inlined into the hot path costs instruction fetch even where it never executes.
+static __device__ __noinline__ void select_fetch_swiglu(const float* __restrict__ gu, int d,
                                                     uint32_t* __restrict__ keys,
                                                     float* __restrict__ x_out) {
   const int tid = threadIdx.x;
@@ -163,7 +165,7 @@ __device__ __forceinline__ void select_fetch_swiglu(const float* __restrict__ gu
 // WINA score keys: keys[j] = bits(|x_j| * norm_j) (one correctly rounded fp32 product; x and
 // the norms read in batches ahead of the arithmetic), the tail of the last quad zero. Ends with
 // a barrier.
-__device__ __forceinline__ void select_fetch_scored(const float* __restrict__ x,
+static __device__ __noinline__ void select_fetch_scored(const float* __restrict__ x,
                                                     const float* __restrict__ norms, int d,
                                                     uint32_t* __restrict__ keys) {
   const int tid = threadIdx.x;
