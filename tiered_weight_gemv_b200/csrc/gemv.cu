@@ -479,7 +479,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
             if (send < nAw) stage_issue(send, min(kBatch2, nAw - send), buf ^ 1);
           }
           const int n = min(todo, send - ka);
-#pragma unroll 2
+#pragma unroll 4
           for (int k = ka; k < ka + n; ++k) decode_approx(k - sbeg, buf);
           ka += n;
           todo -= n;
