@@ -133,7 +133,7 @@ __device__ __forceinline__ void clear_ll4(unsigned long long* p) {
 // Shared memory of the fused kernel ahead of the GEMV's own areas: the selection's scratch and
 // keys share space with the combine and staging areas (they are dead before the GEMV starts).
 __host__ __device__ inline size_t fused_select_bytes(int d) {
-  return (sizeof(SelectSmem) + 15) / 16 * 16 + select_keys_bytes(d) + (size_t(d) + 3) / 4 / 16 * 16 + 16;
+  return (sizeof(SelectSmem) + 15) / 16 * 16 + select_keys_bytes(d);
 }
 
 // FUSED: the kernel first runs the tier rule on x itself (select.cuh: every CTA computes the
@@ -194,8 +194,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
     const uint32_t tf = __float_as_uint(p.prm.t_full) & 0x7FFFFFFFu;
     uint32_t n1, n2;
     bool bad;
-    uint8_t* sgn = reinterpret_cast<uint8_t*>(keys) + select_keys_bytes(p.d_in);
-    select_pass1(p.prm.mode, p.d_in, ts, tf, keys, sel, &n1, &n2, &bad, sgn);
+    select_pass1(p.prm.mode, p.d_in, ts, tf, keys, sel, &n1, &n2, &bad);
     const bool lead = tile == 0 && split == 0;
     if (bad) {  // non-finite x: every tier 0, empty lists, y = 0
       Kf = 0;
@@ -235,9 +234,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
       const int nfl = p.norms ? 0 : min(kGemvMeta, Kf > split ? (Kf - split + S - 1) / S : 0);
       const int nal = p.norms ? 0 : min(kGemvMeta, Ka > split ? (Ka - split + S - 1) / S : 0);
       for (int i = tid; i < nfl; i += kGemvThreads)
-        reinterpret_cast<float*>(meta_col_f)[i] = select_signed_x(keys, sgn, list[split + S * i]);
+        reinterpret_cast<float*>(meta_col_f)[i] = __uint_as_float(keys[list[split + S * i]]);
       for (int i = tid; i < nal; i += kGemvThreads)
-        reinterpret_cast<float*>(meta_col_a)[i] = select_signed_x(keys, sgn, list[a0 + split + S * i]);
+        reinterpret_cast<float*>(meta_col_a)[i] = __uint_as_float(keys[list[a0 + split + S * i]]);
       __syncthreads();  // the keys are dead from here: the GEMV's staging areas reuse them
     }
   } else {

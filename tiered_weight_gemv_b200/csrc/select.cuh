@@ -20,8 +20,9 @@
 // The kernel is bound by instruction issue (a few thousand columns, one CTA), so every pass is a
 // short loop over keys held in shared memory:
 //   fetch    x -> shared memory with cp.async (all loads in flight at once);
-//   pass 1   |x| keys written back, a 4096-bin histogram of key bits 30..19, the threshold counts
-//            (non-finite keys land in the top 16 bins);
+//   pass 1   a 4096-bin histogram of key bits 30..19, the threshold counts (non-finite keys land
+//            in the top 16 bins); x itself stays in shared memory, and every pass clears the sign
+//            bit as it loads a key;
 //   find     a block-wide scan from the top: each boundary's 12-bit bin and the count above it;
 //   pass 2   the keys of those bins: a 1024-bin histogram of bits 18..9 and the sub-bin of rank
 //            K; when rank K is the sub-bin's last key (always, when it holds one key) the sub-bin's
@@ -201,43 +202,36 @@ static __device__ __noinline__ void select_fetch_scored(const float* __restrict_
   __syncthreads();
 }
 
-// Sign bits of quad q's four x values (bit e for x[4q + e]), for select_signed_x.
-__device__ __forceinline__ uint8_t quad_signs(uint4 v) {
-  return (uint8_t)((v.x >> 31) | ((v.y >> 31) << 1) | ((v.z >> 31) << 2) | ((v.w >> 31) << 3));
-}
-// x_j again from its |x| key and the sign bytes pass 1 kept.
-__device__ __forceinline__ float select_signed_x(const uint32_t* keys, const uint8_t* sgn, int j) {
-  return __uint_as_float(keys[j] | ((uint32_t)(sgn[j >> 2] >> (j & 3)) << 31));
+// The |x| keys of quad q: x is kept as it is in shared memory (the product reads its signs back
+// from there), so every pass clears the sign bits as it loads.
+__device__ __forceinline__ uint4 ld_key4(const uint4* kq, int q) {
+  uint4 v = kq[q];
+  v.x &= 0x7FFFFFFFu, v.y &= 0x7FFFFFFFu, v.z &= 0x7FFFFFFFu, v.w &= 0x7FFFFFFFu;
+  return v;
 }
 
-// Pass 1: |x| keys written back, the threshold counts, the non-finite flag and (mode != 0) the
-// 12-bit histogram; sgn (may be null; (d + 3) / 4 bytes) keeps the signs. mode: 0 threshold,
-// 1 TopK, 2 guided. Ends with a barrier; n1, n2 and bad are identical in every thread.
+// Pass 1: the threshold counts, the non-finite flag and (mode != 0) the 12-bit histogram of the
+// |x| keys (x itself stays in keys[]). mode: 0 threshold, 1 TopK, 2 guided. Ends with a barrier;
+// n1, n2 and bad are identical in every thread.
 __device__ __forceinline__ void select_pass1(int mode, int d, uint32_t ts, uint32_t tf,
-                                             uint32_t* __restrict__ keys, SelectSmem& S,
-                                             uint32_t* n1, uint32_t* n2, bool* bad,
-                                             uint8_t* __restrict__ sgn = nullptr) {
+                                             const uint32_t* __restrict__ keys, SelectSmem& S,
+                                             uint32_t* n1, uint32_t* n2, bool* bad) {
   const int tid = threadIdx.x, lane = tid & 31;
   const int nq = (d + 3) >> 2;
-  uint4* kq = reinterpret_cast<uint4*>(keys);
+  const uint4* kq = reinterpret_cast<const uint4*>(keys);
   uint32_t cs = 0, cf = 0, b = 0;
   if (mode == SPAX_MASK_TOPK) {
     for (int q = tid; q < nq; q += kSelThreads) {
-      uint4 v = kq[q];
-      if (sgn) sgn[q] = quad_signs(v);
-      v.x &= 0x7FFFFFFFu, v.y &= 0x7FFFFFFFu, v.z &= 0x7FFFFFFFu, v.w &= 0x7FFFFFFFu;
+      const uint4 v = ld_key4(kq, q);
       atomicAdd(&S.hist[v.x >> 19], 1u);
       atomicAdd(&S.hist[v.y >> 19], 1u);
       atomicAdd(&S.hist[v.z >> 19], 1u);
       atomicAdd(&S.hist[v.w >> 19], 1u);
-      kq[q] = v;
     }
   } else {
     const bool hist = mode == SPAX_MASK_GUIDED;
     for (int q = tid; q < nq; q += kSelThreads) {
-      uint4 v = kq[q];
-      if (sgn) sgn[q] = quad_signs(v);
-      v.x &= 0x7FFFFFFFu, v.y &= 0x7FFFFFFFu, v.z &= 0x7FFFFFFFu, v.w &= 0x7FFFFFFFu;
+      const uint4 v = ld_key4(kq, q);
       cs += (v.x < ts) + (v.y < ts) + (v.z < ts) + (v.w < ts);
       cf += (v.x < tf) + (v.y < tf) + (v.z < tf) + (v.w < tf);
       b = max(b, max(max(v.x, v.y), max(v.z, v.w)));
@@ -247,7 +241,6 @@ __device__ __forceinline__ void select_pass1(int mode, int d, uint32_t ts, uint3
         atomicAdd(&S.hist[v.z >> 19], 1u);
         atomicAdd(&S.hist[v.w >> 19], 1u);
       }
-      kq[q] = v;
     }
     b = b >= 0x7F800000u;
   }
@@ -424,7 +417,7 @@ __device__ __forceinline__ void select_boundaries(const spax_mask_params& prm, i
     const bool same = p0 == p1;
     for (int qb = tid - lane; qb < nq; qb += kSelThreads) {  // warp-uniform trip count
       const int q = qb + lane;
-      const uint4 v = q < nq ? kq[q] : make_uint4(kNoKey, kNoKey, kNoKey, kNoKey);
+      const uint4 v = q < nq ? ld_key4(kq, q) : make_uint4(kNoKey, kNoKey, kNoKey, kNoKey);
       const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -472,7 +465,7 @@ __device__ __forceinline__ void select_boundaries(const spax_mask_params& prm, i
       const bool same2 = q0 == q1;
       for (int qb = tid - lane; qb < nq; qb += kSelThreads) {  // warp-uniform trip count
         const int q = qb + lane;
-        const uint4 v = q < nq ? kq[q] : make_uint4(kNoKey, kNoKey, kNoKey, kNoKey);
+        const uint4 v = q < nq ? ld_key4(kq, q) : make_uint4(kNoKey, kNoKey, kNoKey, kNoKey);
         const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -569,12 +562,12 @@ __device__ __forceinline__ void select_compact(const uint32_t* __restrict__ keys
   // ---- pass 3: counts over the run ----
   uint32_t g0 = 0, g1 = 0, e0 = 0, e1 = 0;
   for (int q = qa; q < qm; ++q) {
-    const uint4 v = kq[q];
+    const uint4 v = ld_key4(kq, q);
     g0 += (v.x >= lo0) + (v.y >= lo0) + (v.z >= lo0) + (v.w >= lo0);
     g1 += (v.x >= lo1) + (v.y >= lo1) + (v.z >= lo1) + (v.w >= lo1);
   }
   if (ragged) {
-    const uint4 v = kq[nfull];
+    const uint4 v = ld_key4(kq, nfull);
     const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -584,7 +577,7 @@ __device__ __forceinline__ void select_compact(const uint32_t* __restrict__ keys
   uint32_t eb0 = 0, eb1 = 0, tot;
   if (ties) {  // keys equal to a boundary key before this run, in column order
     for (int q = qa; q < qb; ++q) {
-      const uint4 v = kq[q];
+      const uint4 v = ld_key4(kq, q);
       const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -610,7 +603,7 @@ __device__ __forceinline__ void select_compact(const uint32_t* __restrict__ keys
   const bool tier_vec = (reinterpret_cast<uintptr_t>(tier) & 3u) == 0;
   if (!ties) {
     for (int q = qa; q < qm; ++q) {
-      const uint4 v = kq[q];
+      const uint4 v = ld_key4(kq, q);
       const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
       uint32_t packed = 0;
 #pragma unroll
@@ -634,7 +627,7 @@ __device__ __forceinline__ void select_compact(const uint32_t* __restrict__ keys
   }
   if (ties || ragged) {  // the general form: bounds checks and ordered equal keys
     for (int q = ties ? qa : qm; q < qb; ++q) {
-      const uint4 v = kq[q];
+      const uint4 v = ld_key4(kq, q);
       const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
