@@ -44,7 +44,6 @@ cudaError_t ensure_smem_limit(const void* kernel, int bytes) {
 }
 
 // Dynamic shared memory a masked GEMV may use (227 KB per CTA, less room for static variables).
-constexpr size_t kMaskedGemvMaxSmem = 227 * 1024 - 1024;
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -233,7 +232,7 @@ static spax_status masked_gemv_common(const spax_packed* W, const float* x, bool
   if (sms < 1) return SPAX_ERR_CUDA;
   GemvPlan pl;
   if (!make_gemv_plan(W->d_out, W->d_in, W->full_fmt, sms, &pl)) return SPAX_ERR_SHAPE;
-  if (masked_gemv_smem_bytes(pl, W->d_in) > kMaskedGemvMaxSmem) return SPAX_ERR_SHAPE;
+  if (masked_gemv_smem_bytes(pl, W->d_in) > kMaskedGemvSmemLimit) return SPAX_ERR_SHAPE;
   if (!ws || ws_bytes < pl.ws_bytes) return SPAX_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(ws) & 255u) return SPAX_ERR_ARG;
   GemvLaunch a;

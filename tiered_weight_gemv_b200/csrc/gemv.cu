@@ -80,6 +80,8 @@ struct GemvParams {
   int32_t* aidx_out;
   int32_t* counts_out;
   int list_bytes;  // 0 for the list-driven kernels
+  int keys_bytes;  // fused: x kept alive after the lists for the product (0: x shares the reused
+                   // area with the GEMV's staging, and the kernel stashes its split's x values)
   int RG;          // row tile R = 512 * RG (1, 2 or 4)
   int swiglu;      // fused only: x holds [g; u] and x_j = swiglu_x(g_j, u_j)
   float* x_out;    // fused swiglu only: the token's x (lead CTA; may be null)
@@ -152,7 +154,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
   int32_t* meta_col_a = reinterpret_cast<int32_t*>(smem);
   int32_t* meta_col_f = meta_col_a + kGemvMeta;
   uint16_t* list = reinterpret_cast<uint16_t*>(meta_col_f + kGemvMeta);  // FUSED: staged lists
-  float* red = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(list) + p.list_bytes);
+  float* red = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(list) + p.list_bytes +
+                                        p.keys_bytes);
+  // fused, keys kept alive: x of every column for the product (null otherwise)
+  const uint32_t* x_live = (FUSED && p.keys_bytes && !p.norms)
+                               ? reinterpret_cast<const uint32_t*>(reinterpret_cast<uint8_t*>(list) +
+                                                                   p.list_bytes)
+                               : nullptr;
   __shared__ int s_bad, s_last;
 
   const int tid = threadIdx.x;
@@ -179,7 +187,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
   if constexpr (FUSED) {
     // ---- the tier rule of this token, computed by every CTA (identical results) ----
     SelectSmem& sel = *reinterpret_cast<SelectSmem*>(red);
-    uint32_t* keys = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(red) +
+    uint32_t* keys = p.keys_bytes ? reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(list) +
+                                                                 p.list_bytes)
+                                  : reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(red) +
                                                  (sizeof(SelectSmem) + 15) / 16 * 16);
     select_zero(sel);
     pdl_wait();
@@ -228,16 +238,18 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
           p.counts_out[3] = p.prm.mode == SPAX_MASK_TOPK ? 0 : (int32_t)n2;
         }
       }
-      // signed x of this split's first kGemvMeta positions of each list, kept in the metadata
-      // arrays (idle in this kernel) for the product: no reload, no recomputation
-      // (not with the WINA score: its keys are scores, so the product reads x itself)
-      const int nfl = p.norms ? 0 : min(kGemvMeta, Kf > split ? (Kf - split + S - 1) / S : 0);
-      const int nal = p.norms ? 0 : min(kGemvMeta, Ka > split ? (Ka - split + S - 1) / S : 0);
-      for (int i = tid; i < nfl; i += kGemvThreads)
-        reinterpret_cast<float*>(meta_col_f)[i] = __uint_as_float(keys[list[split + S * i]]);
-      for (int i = tid; i < nal; i += kGemvThreads)
-        reinterpret_cast<float*>(meta_col_a)[i] = __uint_as_float(keys[list[a0 + split + S * i]]);
-      __syncthreads();  // the keys are dead from here: the GEMV's staging areas reuse them
+      if (!p.keys_bytes) {
+        // x shares the reused area: stash x of this split's first kGemvMeta positions of each
+        // list in the metadata arrays (idle in this kernel) for the product (not with the WINA
+        // score: its keys are scores, so the product reads x itself)
+        const int nfl = p.norms ? 0 : min(kGemvMeta, Kf > split ? (Kf - split + S - 1) / S : 0);
+        const int nal = p.norms ? 0 : min(kGemvMeta, Ka > split ? (Ka - split + S - 1) / S : 0);
+        for (int i = tid; i < nfl; i += kGemvThreads)
+          reinterpret_cast<float*>(meta_col_f)[i] = __uint_as_float(keys[list[split + S * i]]);
+        for (int i = tid; i < nal; i += kGemvThreads)
+          reinterpret_cast<float*>(meta_col_a)[i] = __uint_as_float(keys[list[a0 + split + S * i]]);
+        __syncthreads();  // the keys are dead from here: the GEMV's staging areas reuse them
+      }
     }
   } else {
     pdl_wait();
@@ -294,15 +306,17 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
 
   // x of local position i of this split's approximate / full list: the fused kernel's stash
   // (first kGemvMeta positions), else x of the column
-  const int xs_lim = (FUSED && !p.norms) ? kGemvMeta : 0;  // positions the stash holds
+  const int xs_lim = (FUSED && !p.norms && !p.keys_bytes) ? kGemvMeta : 0;  // stash positions
   auto xA = [&](int i, int col) -> float {
     if constexpr (FUSED) {
+      if (x_live) return __uint_as_float(x_live[col]);
       if (i < xs_lim) return reinterpret_cast<const float*>(meta_col_a)[i];
     }
     return xval(col);
   };
   auto xF = [&](int i, int col) -> float {
     if constexpr (FUSED) {
+      if (x_live) return __uint_as_float(x_live[col]);
       if (i < xs_lim) return reinterpret_cast<const float*>(meta_col_f)[i];
     }
     return xval(col);
@@ -737,11 +751,28 @@ static cudaError_t launch_r(const GemvParams& gp, const GemvPlan& pl, size_t sme
 
 static size_t gemv_smem_bytes() { return kGemvSmemBytes; }
 
-size_t masked_gemv_smem_bytes(const GemvPlan& /*pl: every tile height takes the same*/, int d_in) {
+// Shared memory of the masked GEMV: [metadata][staged lists][x, when it fits][reused area]. The
+// reused area holds the selection's scratch, then the GEMV's combine and staging areas; x sits
+// in it too (and the kernel stashes its split's x values) only when a separate x would not fit.
+// *keys_bytes gets the separate x array's bytes (0: x in the reused area).
+static size_t masked_gemv_layout(int d_in, size_t* keys_bytes) {
   const size_t meta = size_t(2) * kGemvMeta * 4;
   const size_t gemv = gemv_smem_bytes() - meta;  // combine + staging areas
+  const size_t scratch = (sizeof(SelectSmem) + 15) / 16 * 16;
+  const size_t alive = meta + select_list_bytes(d_in) + select_keys_bytes(d_in) +
+                       (gemv > scratch ? gemv : scratch);
+  if (alive <= kMaskedGemvSmemLimit) {
+    *keys_bytes = select_keys_bytes(d_in);
+    return alive;
+  }
   const size_t sel = fused_select_bytes(d_in);
+  *keys_bytes = 0;
   return meta + select_list_bytes(d_in) + (gemv > sel ? gemv : sel);
+}
+
+size_t masked_gemv_smem_bytes(const GemvPlan& /*pl: every tile height takes the same*/, int d_in) {
+  size_t kb;
+  return masked_gemv_layout(d_in, &kb);
 }
 
 static GemvParams make_params(const GemvLaunch& a, const GemvPlan& pl) {
@@ -764,6 +795,7 @@ static GemvParams make_params(const GemvLaunch& a, const GemvPlan& pl) {
   gp.S = pl.S;
   gp.RG = pl.R / 512;
   gp.list_bytes = 0;
+  gp.keys_bytes = 0;
   return gp;
 }
 
@@ -789,7 +821,9 @@ cudaError_t launch_masked_gemv(const GemvLaunch& a, const spax_mask_params& prm,
   gp.aidx_out = approx_idx;
   gp.counts_out = counts;
   gp.list_bytes = (int)select_list_bytes(a.d_in);
-  const size_t smem = masked_gemv_smem_bytes(pl, a.d_in);
+  size_t kb;
+  const size_t smem = masked_gemv_layout(a.d_in, &kb);
+  gp.keys_bytes = (int)kb;
   if (a.full_fmt == SPAX_FULL_BF16) return launch_r<SPAX_FULL_BF16, false, true>(gp, pl, smem, stream);
   return launch_r<SPAX_FULL_INT4_G128, false, true>(gp, pl, smem, stream);
 }

@@ -43,6 +43,8 @@ cudaError_t launch_masked_gemv(const GemvLaunch& a, const spax_mask_params& prm,
                                int32_t* approx_idx, int32_t* counts, const GemvPlan& plan,
                                cudaStream_t stream);
 size_t masked_gemv_smem_bytes(const GemvPlan& plan, int d_in);
+// Dynamic shared memory a masked GEMV may take (227 KB per CTA, less room for static shared).
+constexpr size_t kMaskedGemvSmemLimit = 227 * 1024 - 1024;
 
 cudaError_t launch_mask(const float* x, int d_in, const spax_mask_params& p, uint8_t* tier,
                         int32_t* full_idx, int32_t* approx_idx, int32_t* counts, int32_t* status,

@@ -514,7 +514,9 @@ __device__ __forceinline__ void select_boundaries(const spax_mask_params& prm, i
 }
 
 // Exclusive block-wide prefix of one packed value per thread (two 16-bit fields, totals below
-// 65536), in thread order. Returns the prefix; *total gets the sum. Two barriers.
+// 65536), in thread order. Returns the prefix; *total gets the sum. Two barriers (one with
+// kReuse = false, when nothing writes S.wscan again before the caller's next barrier).
+template <bool kReuse = true>
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, SelectSmem& S, uint32_t* total) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   uint32_t incl = v;
@@ -532,7 +534,7 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, SelectSmem& S, u
     base += w < wid ? s : 0u;
     all += s;
   }
-  __syncthreads();  // S.wscan may be reused right after
+  if (kReuse) __syncthreads();  // S.wscan may be reused right after
   *total = all;
   return base + incl - v;
 }
@@ -592,7 +594,8 @@ __device__ __forceinline__ void select_compact(const uint32_t* __restrict__ keys
     g0 += min(e0, rem0 > eb0 ? rem0 - eb0 : 0u);
     g1 += min(e1, rem1 > eb1 ? rem1 - eb1 : 0u);
   }
-  const uint32_t ex = block_excl_scan(g0 | ((g1 - g0) << 16), S, &tot);
+  // the last scan of the selection: nothing writes S.wscan before the closing barrier below
+  const uint32_t ex = block_excl_scan<false>(g0 | ((g1 - g0) << 16), S, &tot);
   const uint32_t nf = tot & 0xFFFFu, na = tot >> 16, a0 = (nf + 3u) & ~3u;
   *n_full = nf;
   *n_approx = na;
