@@ -466,11 +466,34 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
     if constexpr (FMT == SPAX_FULL_BF16) {
       // bf16 batches of U columns interleaved with 2-bit columns, so the dequant work of the
       // 2-bit tier runs while the bf16 loads are in flight
-      const int per_it = nFw > 0 ? (nAw * U + nFw - 1) / nFw : nAw;
+      // A last round of only 1-2 columns would cost the warp a memory round trip of its own; when
+      // staging buffer 1 is idle (one 2-bit batch at most), those columns are fetched into it by
+      // cp.async at once and added at the end. Only when the split's lists fit one chunk, so the
+      // masked and the list-driven kernels take the same decision (the same order of sums).
+      int ntail = 0;
+      if (max(nf, na) <= kGemvMeta) {
+        const int rounds = (nFw + U - 1) / U, last = nFw - U * (rounds - 1);
+        if (rounds >= 2 && last <= 2 && nAw <= kBatch2) ntail = last;
+      }
+      const int nFr = nFw - ntail;  // columns through registers
+      if (ntail) {
+        __syncwarp();
+        const uint32_t dst = stage_s + kStage2Bytes;  // buffer 1: 1 KB per column, 16 B per chunk
+        for (int q = lane; q < 64 * ntail; q += 32) {
+          const int t = q >> 6, c = q & 63;  // chunk c holds rows rb + 8c .. rb + 8c + 7
+          const int col = max(colF(cg + CG * (nFr + t)), 0);
+          if (rb + 8 * c < p.d_out)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + 1024 * t + 16 * c),
+                         "l"(p.full + col * p.full_col_stride + 2LL * rb + 16 * c)
+                         : "memory");
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+      }
+      const int per_it = nFr > 0 ? (nAw * U + nFr - 1) / nFr : nAw;
       int ka = 0, kf = 0, sbeg = 0, send = 0, buf = 0;
       if (nAw > 0) stage_issue(0, min(kBatch2, nAw), 0);  // on its way before the first bf16 loads
-      while (ka < nAw || kf < nFw) {
-        const int nfb = max(0, min(U, nFw - kf));
+      while (ka < nAw || kf < nFr) {
+        const int nfb = max(0, min(U, nFr - kf));
         uint4 w0[U], w1[U];
         float xf[U];
 #pragma unroll
@@ -482,7 +505,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
           w0[u] = (u < nfb && v0) ? ld_stream128(src) : make_uint4(0u, 0u, 0u, 0u);
           w1[u] = (u < nfb && v1) ? ld_stream128(src + 512) : make_uint4(0u, 0u, 0u, 0u);
         }
-        int todo = (kf + nfb < nFw) ? min(per_it, nAw - ka) : nAw - ka;
+        int todo = (kf + nfb < nFr) ? min(per_it, nAw - ka) : nAw - ka;
         while (todo > 0) {
           if (ka == send) {  // the batch at ka is in flight: wait, then send the next one
             sbeg = ka;
@@ -510,6 +533,25 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
           acc[7] = ffma2(bf16x2_to_f2(w1[u].w), x2, acc[7]);
         }
         kf += nfb;
+      }
+      if (ntail) {  // the tail columns, from buffer 1
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        __syncwarp();
+        for (int t = 0; t < ntail; ++t) {
+          const int i = cg + CG * (nFr + t), col = colF(i);
+          const f2 x2{col >= 0 ? xF(i, col) : 0.f, col >= 0 ? xF(i, col) : 0.f};
+          const uint32_t src = stage_s + kStage2Bytes + 1024 * t + 16 * lane;
+          const uint4 a = v0 ? lds128(src) : make_uint4(0u, 0u, 0u, 0u);
+          const uint4 b = v1 ? lds128(src + 512) : make_uint4(0u, 0u, 0u, 0u);
+          acc[0] = ffma2(bf16x2_to_f2(a.x), x2, acc[0]);
+          acc[1] = ffma2(bf16x2_to_f2(a.y), x2, acc[1]);
+          acc[2] = ffma2(bf16x2_to_f2(a.z), x2, acc[2]);
+          acc[3] = ffma2(bf16x2_to_f2(a.w), x2, acc[3]);
+          acc[4] = ffma2(bf16x2_to_f2(b.x), x2, acc[4]);
+          acc[5] = ffma2(bf16x2_to_f2(b.y), x2, acc[5]);
+          acc[6] = ffma2(bf16x2_to_f2(b.z), x2, acc[6]);
+          acc[7] = ffma2(bf16x2_to_f2(b.w), x2, acc[7]);
+        }
       }
     } else {
       for (int ka = 0; ka < nAw; ka += kBatch2) {
