@@ -18,10 +18,11 @@
 //     CTA's share. Lane l owns rows 8l..8l+7 and 256+8l..256+8l+7 in all three formats, so bf16,
 //     int4 and 2-bit contributions land in the same 16 fp32 accumulators. Weights stream straight
 //     into registers with 16-byte loads marked evict-first, U bf16 columns in flight per warp;
-//     the small 2-bit and int4 records are staged per warp in shared memory, a batch of 16-32
-//     columns at a time. (Measured on B200: one-warp-issued 1-D bulk copies of 0.1-4 KB column
-//     segments are issue-bound at 0.5-3 TB/s; plain 16-byte loads from many warps reach
-//     6.4-6.9 TB/s.)
+//     the small 2-bit records come by cp.async into a per-warp double buffer in shared memory,
+//     a batch of 16 columns sent one batch ahead (int4 records are staged synchronously). A
+//     warp's short last bf16 round is fetched into the idle second buffer with the first loads.
+//     (Measured on B200: one-warp-issued 1-D bulk copies of 0.1-4 KB column segments are
+//     issue-bound at 0.5-3 TB/s; plain 16-byte loads from many warps reach 6.4-6.9 TB/s.)
 //   * 2-bit and int4 codes become floats with one LOP3 each: the code is masked into the
 //     mantissa of a power-of-two constant C (value C + q exactly), multiplied by x_j*scale and
 //     the constant's contribution C*Σ x_j*scale is removed once per row at the end.
