@@ -58,7 +58,8 @@ FALLBACK_HBM_GBS = 6650.0
 def workload_config(tokens: int, replicas: int, world: int) -> dict:
     """The workload description both arms print (the reference arm times a sample of it)."""
     return {"workload": WORKLOAD, "tokens_per_step": tokens,
-            "tiers": {"skip": SKIP, "approx": APPROX, "full": FULL, "rule": "topk"},
+            "tiers": {"skip": SKIP, "approx": APPROX, "full": FULL, "rule": "topk",
+                      "boundary_guess": f"|x| quantiles calibrated on {N_CAL} separate tokens"},
             "weight_replicas": replicas,
             "l2": "inputs larger than L2: each token reads one of the weight replicas",
             "parallelism": f"replicas x{world}"}
@@ -173,15 +174,42 @@ def make_weights(device):
             "gate_up": torch.cat([W["gate"], W["up"]], 0).contiguous(), "down": W["down"]}
 
 
-def make_inputs(mats, n_tokens, device):
+def make_inputs(mats, n_tokens, device, seed=0):
     from tiered_weight_gemv_b200 import synth
     xs = {}
     for name, d_out, d_in, tid in SITES:
         if tid is not None:
-            xs[name] = synth.laplace((n_tokens, d_in), 0, tid, device=device)
+            xs[name] = synth.laplace((n_tokens, d_in), seed, tid, device=device)
     gu = mats["gate_up"].to(torch.float64) @ xs["gate_up"].to(torch.float64).T  # [2*INTER, T]
     xs["down"] = synth.silu_gated(gu[:INTER].T, gu[INTER:].T).contiguous()
     return xs
+
+
+N_CAL = 16  # calibration tokens per site: their own seed, never the timed tokens
+
+
+def calibrated_guesses(mats, device):
+    """Per site, the |x| quantiles at the skip and skip-or-approximate fractions of the TopK
+    counts (spax_calibrate_thresholds over N_CAL separate tokens): the TopK rule takes them in
+    t_skip / t_full as a guess of its boundary keys, which changes how fast the kernels find the
+    boundaries but never which columns they select."""
+    from tiered_weight_gemv_b200 import spax
+    cal = make_inputs(mats, N_CAL, device, seed=1)
+    out = {}
+    for name, d_out, d_in, _ in SITES:
+        kf, ka = k_counts(d_in)
+        ws = torch.empty(spax.spax_workspace_bytes(spax.OP_CALIBRATE, 0, d_in), dtype=torch.uint8,
+                         device=device)
+        t = torch.empty(2, device=device)
+        st = torch.zeros(1, dtype=torch.int32, device=device)
+        spax.spax_calibrate_thresholds(cal[name], round((d_in - kf - ka) * 10000 / d_in),
+                                       round((d_in - kf) * 10000 / d_in), t, st, ws)
+        torch.cuda.synchronize()
+        if int(st.item()) != 0:
+            raise RuntimeError(f"calibration status {int(st.item())} at site {name}")
+        out[name] = tuple(float(v) for v in t.cpu())  # (t_skip, t_full)
+    del cal
+    return out
 
 
 def fused_bytes(d_out, d_in, kf, ka):
@@ -227,6 +255,7 @@ def run_gpu(args, rank, world, local):
     SEL = [s for s in SITES if not args.sites or s[0] in args.sites.split(",")]
     mats = make_weights(dev)
     xs = make_inputs(mats, n_tok, dev)
+    guess = calibrated_guesses(mats, dev)
     host = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         host = ({n: m.cpu() for n, m in mats.items()}, {n: v.cpu() for n, v in xs.items()})
@@ -255,7 +284,9 @@ def run_gpu(args, rank, world, local):
             status=torch.zeros(1, dtype=torch.int32, device=dev),
             ws=spax.alloc_workspace(spax.OP_TIERED_GEMV, d_out, d_in, device=dev),
             dws=spax.alloc_workspace(spax.OP_DENSE_GEMV, d_out, d_in, device=dev),
-            prm=spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka),
+            prm=spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka, t_skip=guess[name][0],
+                                 t_full=guess[name][1]),
+            prm_unguessed=spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka),
             desc=[pm.desc() for pm in packed[name]],
             kf=kf, ka=ka)
 
@@ -274,14 +305,14 @@ def run_gpu(args, rank, world, local):
                                           b["counts"][t], b["y"][t], b["status"], b["ws"],
                                           desc=b["desc"][t % n_rep])
 
-    def step_fused(sites=None):
+    def step_fused(sites=None, prm="prm"):
         """The headline step: one spax_masked_gemv per token and site (mask outputs written)."""
         for t in range(n_tok):
             for name, d_out, d_in, _ in SEL:
                 if sites is not None and name not in sites:
                     continue
                 b = buf[name]
-                spax.spax_masked_gemv(packed[name][t % n_rep], xs[name][t], b["prm"], b["y"][t],
+                spax.spax_masked_gemv(packed[name][t % n_rep], xs[name][t], b[prm], b["y"][t],
                                       b["status"], b["ws"], tier=b["tier"][t],
                                       full_idx=b["fidx"][t], approx_idx=b["aidx"][t],
                                       counts=b["counts"][t], desc=b["desc"][t % n_rep])
@@ -329,6 +360,7 @@ def run_gpu(args, rank, world, local):
         return g
 
     graphs["fused"] = capture(step_fused)
+    graphs["fused_unguessed"] = capture(step_fused, prm="prm_unguessed")
     graphs["tiered"] = capture(step_tiered)
     graphs["dense"] = capture(step_dense)
     graphs["chained"] = capture(step_chained)
@@ -342,6 +374,8 @@ def run_gpu(args, rank, world, local):
     sampler = ClockSampler(local)
     with sampler:
         res["fused"] = max_over_ranks(time_graph(graphs["fused"], args.steps, args.warmup, stream))
+        res["fused_unguessed"] = max_over_ranks(
+            time_graph(graphs["fused_unguessed"], args.steps, args.warmup, stream))
         res["tiered"] = max_over_ranks(time_graph(graphs["tiered"], args.steps, args.warmup, stream))
         res["dense"] = max_over_ranks(time_graph(graphs["dense"], args.steps, args.warmup, stream))
         res["chained"] = max_over_ranks(time_graph(graphs["chained"], args.steps, args.warmup, stream))
@@ -846,6 +880,9 @@ def main():
             "dense_effective_GBps": round(dense_bytes / (res["dense"] * 1e-3) / 1e9, 1),
             "speedup_vs_dense": round(dense / value, 3),
             "two_call_us_per_token_layer": round(two_call, 3),
+            "unguessed_us_per_token_layer": round(us_per_token_layer(res["fused_unguessed"], args.tokens, world), 3),
+            "unguessed_note": "the headline step without the calibrated guess of the TopK boundary "
+                              "keys (same selected columns, found by the full selection)",
             "chained_us_per_token_layer": round(us_per_token_layer(res["chained"], args.tokens, world), 3),
             "chained_note": "down fed from the tiered gate/up output in its own launch "
                             "(spax_masked_gemv_swiglu); informational",

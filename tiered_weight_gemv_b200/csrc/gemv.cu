@@ -201,11 +201,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
       select_fetch_scored(p.x, p.norms, p.d_in, keys);
     else
       select_fetch(p.x, p.d_in, keys);
-    const uint32_t ts = __float_as_uint(p.prm.t_skip) & 0x7FFFFFFFu;
-    const uint32_t tf = __float_as_uint(p.prm.t_full) & 0x7FFFFFFFu;
     uint32_t n1, n2;
-    bool bad;
-    select_pass1(p.prm.mode, p.d_in, ts, tf, keys, sel, &n1, &n2, &bad);
+    Boundary B[2];
+    const bool bad = select_rule(p.prm, p.d_in, keys, sel, &n1, &n2, B);
     const bool lead = tile == 0 && split == 0;
     if (bad) {  // non-finite x: every tier 0, empty lists, y = 0
       Kf = 0;
@@ -220,8 +218,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
       }
       __syncthreads();  // the selection's scratch is dead before the combine area reuses it
     } else {
-      Boundary B[2];
-      select_boundaries(p.prm, p.d_in, keys, n1, n2, sel, B);
       uint32_t nfu, nau;
       select_compact(keys, p.d_in, B, sel, lead ? p.tier_out : nullptr, list, &nfu, &nau, &a0);
       Kf = (int)nfu;

@@ -21,12 +21,9 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   pdl_wait();
   pdl_launch_dependents();
   select_fetch(x, d, keys);  // its barrier also orders the zeroing above
-  const uint32_t ts = __float_as_uint(prm.t_skip) & 0x7FFFFFFFu;
-  const uint32_t tf = __float_as_uint(prm.t_full) & 0x7FFFFFFFu;
   uint32_t n1, n2;
-  bool bad;
-  select_pass1(prm.mode, d, ts, tf, keys, S, &n1, &n2, &bad);
-  if (bad) {
+  Boundary B[2];
+  if (select_rule(prm, d, keys, S, &n1, &n2, B)) {
     for (int j = threadIdx.x; j < d; j += kSelThreads) tier[j] = 0;
     if (threadIdx.x == 0) {
       counts[0] = counts[1] = counts[2] = counts[3] = 0;
@@ -34,8 +31,6 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     }
     return;
   }
-  Boundary B[2];
-  select_boundaries(prm, d, keys, n1, n2, S, B);
   uint16_t* list = reinterpret_cast<uint16_t*>(keys + 4 * ((d + 3) / 4));
   uint32_t nf, na, a0;
   select_compact(keys, d, B, S, tier, list, &nf, &na, &a0);

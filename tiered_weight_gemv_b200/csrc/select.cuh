@@ -42,6 +42,8 @@ constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kSelBins = 4096;            // key bits 30..19
 constexpr uint32_t kNoKey = 0xFFFFFFFFu;  // equal to no finite key
 constexpr uint32_t kNoLo = 0x80000000u;   // above every finite key
+constexpr int kSelCand = 32;              // keys of one window bin a guessed boundary ranks
+constexpr int kSelGuessMaxD = 8192;       // widest x the guessed TopK search takes (below)
 
 struct Boundary {
   uint32_t lo, eqv, rem;
@@ -55,7 +57,9 @@ struct SelectSmem {
   uint32_t sel[2][4];    // per boundary: prefix / key, count above, count in the bin
   alignas(16) uint32_t wsum[kSelWarps];
   alignas(16) uint32_t wscan[kSelWarps];
-  uint32_t flag[2];
+  uint32_t hint[8];           // guessed TopK: #keys above each window (0, 2), the largest key
+                              // (4), the keys gathered from one bin per boundary (5, 6)
+  uint32_t cand[2][kSelCand]; // guessed TopK: those gathered keys
 };
 
 // Dynamic shared memory the keys of d columns take (padded to whole 16-byte quads).
@@ -84,6 +88,7 @@ __device__ __forceinline__ void select_zero(SelectSmem& S) {
   for (int i = threadIdx.x; i < 2 * 1024; i += kSelThreads) (&S.ha[0][0])[i] = 0u;
   for (int i = threadIdx.x; i < 2 * 512; i += kSelThreads) (&S.hb[0][0])[i] = 0u;
   if (threadIdx.x < 4) S.stat[threadIdx.x] = 0u;
+  if (threadIdx.x < 8) S.hint[threadIdx.x] = 0u;
 }
 
 // x[0, d) -> keys[] as raw fp32 bits; the tail of the last quad is zero. Ends with a barrier.
@@ -511,6 +516,193 @@ __device__ __forceinline__ void select_boundaries(const spax_mask_params& prm, i
       B[t].rem = 0u;
     }
   }
+}
+
+// The window of a guess h of a boundary key: keys [lo, lo + (1024 << sh)), lo the key of 7h/8
+// and the span reaching at least to the key of 9h/8 (at most 2^23 keys: the two values are less
+// than a factor 2 apart). False when h is not a positive finite number or 7h/8 rounds to zero.
+__device__ __forceinline__ bool guess_window(float h, uint32_t* lo, int* sh) {
+  if (__float_as_uint(h) - 1u >= 0x7F7FFFFFu) return false;  // NaN, Inf, negative or zero
+  const uint32_t a = __float_as_uint(h * 0.875f), b = __float_as_uint(h * 1.125f);
+  if (a == 0u) return false;
+  const uint32_t r = b - a;
+  *lo = a;
+  *sh = r <= 1024u ? 0 : 32 - __clz((r - 1u) >> 10);
+  return true;
+}
+
+// TopK boundaries found from a guess of each boundary key: the calibrated thresholds a caller may
+// pass in t_full (boundary 0) and t_skip (boundary 1), which the TopK rule has no other use for.
+// One pass over the keys counts, per boundary, the keys above a window around its guess and
+// histograms the keys inside it (1024 bins of 2^sh keys). When each rank K lies inside its window,
+// a block scan of the histograms gives the bin of rank K; where that bin also holds keys ranked
+// after K its keys are gathered and ranked among themselves. Returns 1 when B is set, 2 on a
+// non-finite key (B unset), 0 when the guesses do not apply or miss, or a bin is too crowded to
+// rank (S.ha is zero again then, S.hist untouched: the unhinted selection follows). The guess
+// decides only how the boundaries are found: B describes the same two sets either way.
+// All threads; barriers inside.
+__device__ __forceinline__ int select_topk_guessed(const spax_mask_params& prm, int d,
+                                                   const uint32_t* __restrict__ keys,
+                                                   SelectSmem& S, Boundary* B) {
+  const uint32_t K0 = (uint32_t)prm.k_full, K1 = (uint32_t)prm.k_full + (uint32_t)prm.k_approx;
+  const bool act0 = K0 > 0u && K0 < (uint32_t)d, act1 = K1 > 0u && K1 < (uint32_t)d;
+  uint32_t lo0 = 0u, lo1 = 0u;
+  int sh0 = 0, sh1 = 0;
+  if (d > kSelGuessMaxD || (!act0 && !act1)) return 0;
+  if (act0 && !guess_window(prm.t_full, &lo0, &sh0)) return 0;
+  if (act1 && !guess_window(prm.t_skip, &lo1, &sh1)) return 0;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int nq = (d + 3) >> 2;
+  const uint4* kq = reinterpret_cast<const uint4*>(keys);
+  // ---- one pass: keys above each window, the window histograms, the largest key. The zero
+  // keys padding the last quad lie below every window (lo >= 1) and count nowhere. ----
+  const uint32_t w0 = act0 ? (1024u << sh0) : 0u, w1 = act1 ? (1024u << sh1) : 0u;
+  const uint32_t hi0 = lo0 + w0, hi1 = lo1 + w1;
+  if (tid < 2) S.sel[tid][0] = kNoKey;  // stays when rank K is outside the window (a miss)
+  uint32_t a0 = 0, a1 = 0, mx = 0;
+  for (int q = tid; q < nq; q += kSelThreads) {
+    const uint4 v = ld_key4(kq, q);
+    const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t k = kk[e], r0 = k - lo0, r1 = k - lo1;
+      mx = max(mx, k);
+      a0 += k >= hi0;
+      a1 += k >= hi1;
+      if (r0 < w0) atomicAdd(&S.ha[0][r0 >> sh0], 1u);
+      if (r1 < w1) atomicAdd(&S.ha[1][r1 >> sh1], 1u);
+    }
+  }
+  a0 = __reduce_add_sync(0xffffffffu, a0);
+  a1 = __reduce_add_sync(0xffffffffu, a1);
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  if (lane == 0) {
+    atomicAdd(&S.hint[0], a0);
+    atomicAdd(&S.hint[2], a1);
+    atomicMax(&S.hint[4], mx);
+  }
+  __syncthreads();
+  if (S.hint[4] >= 0x7F800000u) return 2;  // Inf / NaN among the keys
+  const uint32_t A0 = S.hint[0], A1 = S.hint[2];
+  auto unwind = [&]() {  // a miss: the unhinted selection needs S.ha zero
+    for (int i = tid; i < 2 * 1024; i += kSelThreads) (&S.ha[0][0])[i] = 0u;
+    return 0;
+  };
+  // rank K lies in the window iff the scan from the top finds it before the window's bottom
+  block_find_pair<1024>(S.ha[0], S.ha[1], act0, act1, K0, K1, A0, A1, 0u, 0u, 0, S);
+  if ((act0 && S.sel[0][0] == kNoKey) || (act1 && S.sel[1][0] == kNoKey)) return unwind();
+  // ---- per boundary: the bin of rank K, the count above it and in it ----
+  uint32_t base[2], above[2], cnt[2];
+  bool need[2];
+  bool crowded = false;
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const uint32_t K = t ? K1 : K0;
+    need[t] = false;
+    base[t] = above[t] = cnt[t] = 0u;
+    if (!(t ? act1 : act0)) {
+      B[t].lo = K ? 0u : kNoLo;  // K = d: every column; K = 0: none
+      B[t].eqv = kNoKey;
+      B[t].rem = 0u;
+      continue;
+    }
+    const int sh = t ? sh1 : sh0;
+    base[t] = (t ? lo1 : lo0) + (S.sel[t][0] << sh);
+    above[t] = S.sel[t][1];
+    cnt[t] = S.sel[t][2];
+    const uint32_t rem = K - above[t];
+    if (rem == cnt[t]) {  // the whole bin is in: its lower edge bounds the set
+      B[t].lo = base[t];
+      B[t].eqv = kNoKey;
+      B[t].rem = 0u;
+    } else if (sh == 0) {  // a one-key bin: that key, and rem of its cnt copies
+      B[t].lo = base[t] + 1u;
+      B[t].eqv = base[t];
+      B[t].rem = rem;
+    } else {
+      need[t] = true;
+      crowded |= cnt[t] > (uint32_t)kSelCand;
+    }
+  }
+  if (!need[0] && !need[1]) return 1;
+  if (crowded) return unwind();
+  // ---- gather the keys of each unresolved bin, then rank them (one warp per boundary) ----
+  const uint32_t g0 = base[0], g1 = base[1];
+  const uint32_t gw0 = need[0] ? (1u << sh0) : 0u, gw1 = need[1] ? (1u << sh1) : 0u;
+  for (int q = tid; q < nq; q += kSelThreads) {
+    const uint4 v = ld_key4(kq, q);
+    const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (kk[e] - g0 < gw0) {
+        const uint32_t i = atomicAdd(&S.hint[5], 1u);
+        if (i < (uint32_t)kSelCand) S.cand[0][i] = kk[e];
+      }
+      if (kk[e] - g1 < gw1) {
+        const uint32_t i = atomicAdd(&S.hint[6], 1u);
+        if (i < (uint32_t)kSelCand) S.cand[1][i] = kk[e];
+      }
+    }
+  }
+  __syncthreads();
+  // the gathered counts equal the histogram's by construction; anything else is not trusted
+  if ((need[0] && S.hint[5] != cnt[0]) || (need[1] && S.hint[6] != cnt[1])) return unwind();
+  const int wid = tid >> 5;
+  if (wid < 2 && (wid ? need[1] : need[0])) {  // warp t ranks boundary t's keys: V, gt < rem <= gt + eq
+    const uint32_t c = wid ? cnt[1] : cnt[0], ab = wid ? above[1] : above[0];
+    const uint32_t rem = (wid ? K1 : K0) - ab;
+    const uint32_t v = (uint32_t)lane < c ? S.cand[wid][lane] : kNoKey;
+    uint32_t gt = 0, eq = 0;
+    for (uint32_t j = 0; j < c; ++j) {
+      const uint32_t u = __shfl_sync(0xffffffffu, v, (int)j);
+      gt += u > v;
+      eq += u == v;
+    }
+    // S.sel was read into registers before the barrier above
+    if ((uint32_t)lane < c && gt < rem && rem <= gt + eq) {
+      S.sel[wid][0] = v;
+      S.sel[wid][1] = ab + gt;
+      S.sel[wid][2] = eq;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    if (!need[t]) continue;
+    const uint32_t V = S.sel[t][0], rem = (t ? K1 : K0) - S.sel[t][1], eq = S.sel[t][2];
+    if (rem == eq) {
+      B[t].lo = V;
+      B[t].eqv = kNoKey;
+      B[t].rem = 0u;
+    } else {
+      B[t].lo = V + 1u;
+      B[t].eqv = V;
+      B[t].rem = rem;
+    }
+  }
+  return 1;
+}
+
+// The rule's two boundaries (after a select_fetch*; all threads; barriers inside): the guessed
+// TopK search when it applies and resolves, else pass 1 and select_boundaries. Returns true on a
+// non-finite key (B unset). n1, n2: the threshold counts (0 in TopK mode).
+__device__ __forceinline__ bool select_rule(const spax_mask_params& prm, int d,
+                                            const uint32_t* __restrict__ keys, SelectSmem& S,
+                                            uint32_t* n1, uint32_t* n2, Boundary* B) {
+  if (prm.mode == SPAX_MASK_TOPK) {
+    const int g = select_topk_guessed(prm, d, keys, S, B);
+    if (g != 0) {
+      *n1 = *n2 = 0u;
+      return g == 2;
+    }
+  }
+  const uint32_t ts = __float_as_uint(prm.t_skip) & 0x7FFFFFFFu;
+  const uint32_t tf = __float_as_uint(prm.t_full) & 0x7FFFFFFFu;
+  bool bad;
+  select_pass1(prm.mode, d, ts, tf, keys, S, n1, n2, &bad);
+  if (bad) return true;
+  select_boundaries(prm, d, keys, *n1, *n2, S, B);
+  return false;
 }
 
 // Exclusive block-wide prefix of one packed value per thread (two 16-bit fields, totals below
