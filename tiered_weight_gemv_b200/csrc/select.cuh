@@ -560,6 +560,8 @@ __device__ __forceinline__ int select_topk_guessed(const spax_mask_params& prm, 
   const uint32_t hi0 = lo0 + w0, hi1 = lo1 + w1;
   if (tid < 2) S.sel[tid][0] = kNoKey;  // stays when rank K is outside the window (a miss)
   uint32_t a0 = 0, a1 = 0, mx = 0;
+  // disjoint windows (the usual case): one atomic per key, into whichever window holds it
+  const bool disjoint = hi0 <= lo1 || hi1 <= lo0;
   for (int q = tid; q < nq; q += kSelThreads) {
     const uint4 v = ld_key4(kq, q);
     const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
@@ -569,8 +571,13 @@ __device__ __forceinline__ int select_topk_guessed(const spax_mask_params& prm, 
       mx = max(mx, k);
       a0 += k >= hi0;
       a1 += k >= hi1;
-      if (r0 < w0) atomicAdd(&S.ha[0][r0 >> sh0], 1u);
-      if (r1 < w1) atomicAdd(&S.ha[1][r1 >> sh1], 1u);
+      const bool in0 = r0 < w0, in1 = r1 < w1;
+      if (disjoint) {
+        if (in0 || in1) atomicAdd(in0 ? &S.ha[0][r0 >> sh0] : &S.ha[1][r1 >> sh1], 1u);
+      } else {
+        if (in0) atomicAdd(&S.ha[0][r0 >> sh0], 1u);
+        if (in1) atomicAdd(&S.ha[1][r1 >> sh1], 1u);
+      }
     }
   }
   a0 = __reduce_add_sync(0xffffffffu, a0);
