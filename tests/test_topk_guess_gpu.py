@@ -3,7 +3,7 @@ skipped): the guess only changes how the kernels find the boundaries, never the 
 case compares the mask's tiers, lists and counts with the oracle bit for bit, and the one-launch
 masked GEMV with and without the guess bit for bit.
 
-`guess_path` restates, on the host, how the kernels use a guess (a window of 1024 bins around it,
+`guess_path` restates, on the host, how the kernels use a guess (a window of 2048 bins around it,
 the bin of rank K, the keys of that bin), so each case can assert which branch it exercises: a
 miss, a whole bin, a one-key bin, a gathered bin, a bin too crowded to rank, or an invalid guess.
 """
@@ -20,6 +20,7 @@ pytestmark = pytest.mark.gpu
 
 CAND = 32  # keys of one bin the kernels rank; more falls back to the full selection
 MAX_D = 8192  # widest x the kernels search with a guess; wider x always takes the full selection
+BINS = 2048  # bins of one window
 
 
 def _f32(v) -> np.float32:
@@ -27,7 +28,7 @@ def _f32(v) -> np.float32:
 
 
 def window(h):
-    """(lo, sh) of a guess h, or None when h is not usable (keys [lo, lo + (1024 << sh)))."""
+    """(lo, sh) of a guess h, or None when h is not usable (keys [lo, lo + (BINS << sh)))."""
     hb = int(np.array([h], np.float32).view(np.uint32)[0])
     if not 1 <= hb <= 0x7F7FFFFF:
         return None
@@ -36,7 +37,7 @@ def window(h):
     if a == 0:
         return None
     r = b - a
-    return a, (0 if r <= 1024 else ((r - 1) >> 10).bit_length())
+    return a, (0 if r <= BINS else ((r - 1) // BINS).bit_length())
 
 
 def guess_path(x: np.ndarray, K: int, h) -> str:
@@ -51,14 +52,14 @@ def guess_path(x: np.ndarray, K: int, h) -> str:
     if w is None:
         return "invalid"
     lo, sh = w
-    hi = lo + (1024 << sh)
+    hi = lo + (BINS << sh)
     A = int(np.sum(keys >= hi))
     inside = keys[(keys >= lo) & (keys < hi)]
     if not (A < K <= A + inside.size):
         return "miss"
-    cnt = np.bincount((inside - lo) >> sh, minlength=1024)
+    cnt = np.bincount((inside - lo) >> sh, minlength=BINS)
     above = A
-    for b in range(1023, -1, -1):
+    for b in range(BINS - 1, -1, -1):
         if above < K <= above + cnt[b]:
             rem, c = K - above, int(cnt[b])
             if rem == c:
@@ -116,7 +117,7 @@ def _clustered(d, seed):
 
 
 def _subnormal(d, seed):
-    """Subnormal magnitudes (bit patterns 1..3000, random signs): windows of 1024 single-key bins."""
+    """Subnormal magnitudes (bit patterns 1..3000, random signs): windows of single-key bins."""
     rng = np.random.default_rng(seed)
     bits = rng.integers(1, 3000, d).astype(np.uint32) | (rng.integers(0, 2, d).astype(np.uint32) << 31)
     return bits.view(np.float32).copy()
@@ -144,7 +145,9 @@ def test_guess_laplace_all_branches(d):
             seen.add(guess_path(x, kf + ka, ts))
             m.check(x, kf, ka, tf, ts, f"d={d} kf={kf} ka={ka} scale={scale}")
     if 1000 <= d <= MAX_D:
-        assert {"miss", "bin", "gather"} <= seen, seen
+        assert {"miss", "bin"} <= seen, seen
+    if d in (1000, 4096):
+        assert "gather" in seen, seen
 
 
 def test_guess_invalid_and_edge_values():

@@ -44,6 +44,8 @@ constexpr uint32_t kNoKey = 0xFFFFFFFFu;  // equal to no finite key
 constexpr uint32_t kNoLo = 0x80000000u;   // above every finite key
 constexpr int kSelCand = 32;              // keys of one window bin a guessed boundary ranks
 constexpr int kSelGuessMaxD = 8192;       // widest x the guessed TopK search takes (below)
+constexpr int kGuessBins = 2048;          // bins of one guessed window (two windows fill hist)
+static_assert(2 * kGuessBins <= kSelBins && kGuessBins == 1 << 11, "window bins");
 
 struct Boundary {
   uint32_t lo, eqv, rem;
@@ -518,29 +520,30 @@ __device__ __forceinline__ void select_boundaries(const spax_mask_params& prm, i
   }
 }
 
-// The window of a guess h of a boundary key: keys [lo, lo + (1024 << sh)), lo the key of 7h/8
-// and the span reaching at least to the key of 9h/8 (at most 2^23 keys: the two values are less
-// than a factor 2 apart). False when h is not a positive finite number or 7h/8 rounds to zero.
+// The window of a guess h of a boundary key: keys [lo, lo + (kGuessBins << sh)), lo the key of
+// 7h/8 and the span reaching at least to the key of 9h/8 (at most 2^23 keys: the two values are
+// less than a factor 2 apart). False when h is not a positive finite number or 7h/8 rounds to
+// zero.
 __device__ __forceinline__ bool guess_window(float h, uint32_t* lo, int* sh) {
   if (__float_as_uint(h) - 1u >= 0x7F7FFFFFu) return false;  // NaN, Inf, negative or zero
   const uint32_t a = __float_as_uint(h * 0.875f), b = __float_as_uint(h * 1.125f);
   if (a == 0u) return false;
   const uint32_t r = b - a;
   *lo = a;
-  *sh = r <= 1024u ? 0 : 32 - __clz((r - 1u) >> 10);
+  *sh = r <= (uint32_t)kGuessBins ? 0 : 32 - __clz((r - 1u) >> 11);
   return true;
 }
 
 // TopK boundaries found from a guess of each boundary key: the calibrated thresholds a caller may
 // pass in t_full (boundary 0) and t_skip (boundary 1), which the TopK rule has no other use for.
 // One pass over the keys counts, per boundary, the keys above a window around its guess and
-// histograms the keys inside it (1024 bins of 2^sh keys). When each rank K lies inside its window,
-// a block scan of the histograms gives the bin of rank K; where that bin also holds keys ranked
-// after K its keys are gathered and ranked among themselves. Returns 1 when B is set, 2 on a
-// non-finite key (B unset), 0 when the guesses do not apply or miss, or a bin is too crowded to
-// rank (S.ha is zero again then, S.hist untouched: the unhinted selection follows). The guess
-// decides only how the boundaries are found: B describes the same two sets either way.
-// All threads; barriers inside.
+// histograms the keys inside it (kGuessBins bins of 2^sh keys each, the two windows side by side
+// in S.hist). When each rank K lies inside its window, a block scan of the histograms gives the
+// bin of rank K; where that bin also holds keys ranked after K its keys are gathered and ranked
+// among themselves. Returns 1 when B is set, 2 on a non-finite key (B unset), 0 when the guesses
+// do not apply or miss, or a bin is too crowded to rank (S.hist is zero again then: the unhinted
+// selection follows). The guess decides only how the boundaries are found: B describes the same
+// two sets either way. All threads; barriers inside.
 __device__ __forceinline__ int select_topk_guessed(const spax_mask_params& prm, int d,
                                                    const uint32_t* __restrict__ keys,
                                                    SelectSmem& S, Boundary* B) {
@@ -556,7 +559,10 @@ __device__ __forceinline__ int select_topk_guessed(const spax_mask_params& prm, 
   const uint4* kq = reinterpret_cast<const uint4*>(keys);
   // ---- one pass: keys above each window, the window histograms, the largest key. The zero
   // keys padding the last quad lie below every window (lo >= 1) and count nowhere. ----
-  const uint32_t w0 = act0 ? (1024u << sh0) : 0u, w1 = act1 ? (1024u << sh1) : 0u;
+  const uint32_t w0 = act0 ? ((uint32_t)kGuessBins << sh0) : 0u;
+  const uint32_t w1 = act1 ? ((uint32_t)kGuessBins << sh1) : 0u;
+  uint32_t* h0 = S.hist;
+  uint32_t* h1 = S.hist + kGuessBins;
   const uint32_t hi0 = lo0 + w0, hi1 = lo1 + w1;
   if (tid < 2) S.sel[tid][0] = kNoKey;  // stays when rank K is outside the window (a miss)
   uint32_t a0 = 0, a1 = 0, mx = 0;
@@ -573,10 +579,10 @@ __device__ __forceinline__ int select_topk_guessed(const spax_mask_params& prm, 
       a1 += k >= hi1;
       const bool in0 = r0 < w0, in1 = r1 < w1;
       if (disjoint) {
-        if (in0 || in1) atomicAdd(in0 ? &S.ha[0][r0 >> sh0] : &S.ha[1][r1 >> sh1], 1u);
+        if (in0 || in1) atomicAdd(in0 ? &h0[r0 >> sh0] : &h1[r1 >> sh1], 1u);
       } else {
-        if (in0) atomicAdd(&S.ha[0][r0 >> sh0], 1u);
-        if (in1) atomicAdd(&S.ha[1][r1 >> sh1], 1u);
+        if (in0) atomicAdd(&h0[r0 >> sh0], 1u);
+        if (in1) atomicAdd(&h1[r1 >> sh1], 1u);
       }
     }
   }
@@ -591,12 +597,13 @@ __device__ __forceinline__ int select_topk_guessed(const spax_mask_params& prm, 
   __syncthreads();
   if (S.hint[4] >= 0x7F800000u) return 2;  // Inf / NaN among the keys
   const uint32_t A0 = S.hint[0], A1 = S.hint[2];
-  auto unwind = [&]() {  // a miss: the unhinted selection needs S.ha zero
-    for (int i = tid; i < 2 * 1024; i += kSelThreads) (&S.ha[0][0])[i] = 0u;
+  auto unwind = [&]() {  // a miss: the unhinted selection needs S.hist zero
+    for (int i = 4 * tid; i < kSelBins; i += 4 * kSelThreads)
+      *reinterpret_cast<uint4*>(&S.hist[i]) = make_uint4(0u, 0u, 0u, 0u);
     return 0;
   };
   // rank K lies in the window iff the scan from the top finds it before the window's bottom
-  block_find_pair<1024>(S.ha[0], S.ha[1], act0, act1, K0, K1, A0, A1, 0u, 0u, 0, S);
+  block_find_pair<kGuessBins>(h0, h1, act0, act1, K0, K1, A0, A1, 0u, 0u, 0, S);
   if ((act0 && S.sel[0][0] == kNoKey) || (act1 && S.sel[1][0] == kNoKey)) return unwind();
   // ---- per boundary: the bin of rank K, the count above it and in it ----
   uint32_t base[2], above[2], cnt[2];
