@@ -88,9 +88,9 @@ typedef enum { SPAX_OP_TIERED_GEMV = 0, SPAX_OP_DENSE_GEMV = 1, SPAX_OP_CALIBRAT
  *     k_full + k_approx <= d_in. t_full and t_skip are an optional guess of the |x| at rank
  *     k_full and at rank k_full + k_approx (calibrated quantiles, e.g. from
  *     spax_calibrate_thresholds at the skip fractions 1 - (k_full + k_approx)/d_in and
- *     1 - k_full/d_in): for d_in <= 8192 a guess within about 12% lets the kernels find the
- *     boundaries in one windowed pass instead of the full search. Any value is accepted (0, a
- *     negative, NaN or Inf means no guess), and the selected columns never depend on it.
+ *     1 - k_full/d_in): a guess within about 12% lets the kernels find the boundaries in one
+ *     windowed pass instead of the full search. Any value is accepted (0, a negative, NaN or
+ *     Inf means no guess), and the selected columns never depend on it.
  *   GUIDED (TopK-Guided §2.1): the natural counts n1 = #{|x| < t_skip} and n2 = #{|x| < t_full}
  *     are clipped into the bands [ceil((s-δ)d), floor((s+δ)d)] around the skip target
  *     s = s_skip_bp/1e4 and the skip-or-approximate target s = s_below_full_bp/1e4

@@ -43,7 +43,6 @@ constexpr int kSelBins = 4096;            // key bits 30..19
 constexpr uint32_t kNoKey = 0xFFFFFFFFu;  // equal to no finite key
 constexpr uint32_t kNoLo = 0x80000000u;   // above every finite key
 constexpr int kSelCand = 32;              // keys of one window bin a guessed boundary ranks
-constexpr int kSelGuessMaxD = 8192;       // widest x the guessed TopK search takes (below)
 constexpr int kGuessBins = 2048;          // bins of one guessed window (two windows fill hist)
 static_assert(2 * kGuessBins <= kSelBins && kGuessBins == 1 << 11, "window bins");
 
@@ -551,7 +550,7 @@ __device__ __forceinline__ int select_topk_guessed(const spax_mask_params& prm, 
   const bool act0 = K0 > 0u && K0 < (uint32_t)d, act1 = K1 > 0u && K1 < (uint32_t)d;
   uint32_t lo0 = 0u, lo1 = 0u;
   int sh0 = 0, sh1 = 0;
-  if (d > kSelGuessMaxD || (!act0 && !act1)) return 0;
+  if (!act0 && !act1) return 0;
   if (act0 && !guess_window(prm.t_full, &lo0, &sh0)) return 0;
   if (act1 && !guess_window(prm.t_skip, &lo1, &sh1)) return 0;
   const int tid = threadIdx.x, lane = tid & 31;
