@@ -287,6 +287,8 @@ def run_gpu(args, rank, world, local):
             prm=spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka, t_skip=guess[name][0],
                                  t_full=guess[name][1]),
             prm_unguessed=spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka),
+            prm_missed=spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka,
+                                        t_skip=2 * guess[name][0], t_full=2 * guess[name][1]),
             desc=[pm.desc() for pm in packed[name]],
             kf=kf, ka=ka)
 
@@ -361,6 +363,7 @@ def run_gpu(args, rank, world, local):
 
     graphs["fused"] = capture(step_fused)
     graphs["fused_unguessed"] = capture(step_fused, prm="prm_unguessed")
+    graphs["fused_missed"] = capture(step_fused, prm="prm_missed")
     graphs["tiered"] = capture(step_tiered)
     graphs["dense"] = capture(step_dense)
     graphs["chained"] = capture(step_chained)
@@ -376,6 +379,8 @@ def run_gpu(args, rank, world, local):
         res["fused"] = max_over_ranks(time_graph(graphs["fused"], args.steps, args.warmup, stream))
         res["fused_unguessed"] = max_over_ranks(
             time_graph(graphs["fused_unguessed"], args.steps, args.warmup, stream))
+        res["fused_missed"] = max_over_ranks(
+            time_graph(graphs["fused_missed"], args.steps, args.warmup, stream))
         res["tiered"] = max_over_ranks(time_graph(graphs["tiered"], args.steps, args.warmup, stream))
         res["dense"] = max_over_ranks(time_graph(graphs["dense"], args.steps, args.warmup, stream))
         res["chained"] = max_over_ranks(time_graph(graphs["chained"], args.steps, args.warmup, stream))
@@ -883,6 +888,10 @@ def main():
             "unguessed_us_per_token_layer": round(us_per_token_layer(res["fused_unguessed"], args.tokens, world), 3),
             "unguessed_note": "the headline step without the calibrated guess of the TopK boundary "
                               "keys (same selected columns, found by the full selection)",
+            "guess_missed_us_per_token_layer": round(us_per_token_layer(res["fused_missed"], args.tokens, world), 3),
+            "guess_missed_note": "the same step with every guess twice the calibrated key, so every "
+                                 "launch misses its windows and then runs the full selection (the "
+                                 "worst case of a wrong guess)",
             "chained_us_per_token_layer": round(us_per_token_layer(res["chained"], args.tokens, world), 3),
             "chained_note": "down fed from the tiered gate/up output in its own launch "
                             "(spax_masked_gemv_swiglu); informational",

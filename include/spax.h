@@ -90,7 +90,9 @@ typedef enum { SPAX_OP_TIERED_GEMV = 0, SPAX_OP_DENSE_GEMV = 1, SPAX_OP_CALIBRAT
  *     spax_calibrate_thresholds at the skip fractions 1 - (k_full + k_approx)/d_in and
  *     1 - k_full/d_in): a guess within about 12% lets the kernels find the boundaries in one
  *     windowed pass instead of the full search. Any value is accepted (0, a negative, NaN or
- *     Inf means no guess), and the selected columns never depend on it.
+ *     Inf means no guess), and the selected columns never depend on it. A guess that misses
+ *     costs that pass (about 1-1.5 us per launch) on top of the full search, so pass none where
+ *     the token-to-token scale of x varies by more than the window.
  *   GUIDED (TopK-Guided §2.1): the natural counts n1 = #{|x| < t_skip} and n2 = #{|x| < t_full}
  *     are clipped into the bands [ceil((s-δ)d), floor((s+δ)d)] around the skip target
  *     s = s_skip_bp/1e4 and the skip-or-approximate target s = s_below_full_bp/1e4
@@ -252,7 +254,8 @@ spax_status spax_masked_gemv(const spax_packed* h_W, const float* d_x,
  * (its per-element score: activation magnitude times the column norm).
  * d_norms: fp32 [d_in] (device), as spax_column_norms writes them. The score is one correctly
  * rounded fp32 product; every rule (threshold, TopK, guided) and tie order of spax_build_mask
- * then applies to s in place of |x| (thresholds are on s). The product still uses x. A
+ * then applies to s in place of |x| (thresholds, and a TopK guess of the boundary keys, are on
+ * s). The product still uses x. A
  * non-finite score is SPAX_ERR_NONFINITE. Every other argument, output and rule as
  * spax_masked_gemv.
  */
