@@ -91,7 +91,7 @@ typedef enum { SPAX_OP_TIERED_GEMV = 0, SPAX_OP_DENSE_GEMV = 1, SPAX_OP_CALIBRAT
  *     1 - k_full/d_in): a guess within about 12% lets the kernels find the boundaries in one
  *     windowed pass instead of the full search. Any value is accepted (0, a negative, NaN or
  *     Inf means no guess), and the selected columns never depend on it. A guess that misses
- *     costs that pass (about 1-1.5 us per launch) on top of the full search, so pass none where
+ *     costs that pass (about 2 us per launch) on top of the full search, so pass none where
  *     the token-to-token scale of x varies by more than the window.
  *   GUIDED (TopK-Guided §2.1): the natural counts n1 = #{|x| < t_skip} and n2 = #{|x| < t_full}
  *     are clipped into the bands [ceil((s-δ)d), floor((s+δ)d)] around the skip target
