@@ -31,6 +31,8 @@
 //   pass 3   per-thread counts over a contiguous run of columns, one block scan;
 //   pass 4   tier codes and the ascending lists (staged in shared memory, then copied out with
 //            16-byte stores), written from the same runs.
+// With a TopK guess of the two boundary keys (select_topk_guessed), one windowed pass and a
+// 2048-bin scan per boundary take the place of passes 1 to 2b whenever the guess holds.
 #pragma once
 
 #include "common.cuh"
