@@ -233,6 +233,9 @@ def spax_calibrate_thresholds(calib_x: torch.Tensor, s_skip_bp: int, s_below_ful
 
 def mask_params(mode: int, *, t_skip=0.0, t_full=0.0, k_full=0, k_approx=0, s_skip_bp=0,
                 s_below_full_bp=0, delta_bp=0) -> spax_mask_params:
+    """The rule's parameters (spax.h, spax_mask_params). In MASK_TOPK mode t_full / t_skip may
+    carry a guess of the |x| at rank k_full / k_full + k_approx (calibrated quantiles); it only
+    speeds the selection up when it holds, and 0 means no guess."""
     return spax_mask_params(mode, t_skip, t_full, k_full, k_approx, s_skip_bp, s_below_full_bp,
                             delta_bp)
 
