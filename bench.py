@@ -307,14 +307,17 @@ def run_gpu(args, rank, world, local):
                                           b["counts"][t], b["y"][t], b["status"], b["ws"],
                                           desc=b["desc"][t % n_rep])
 
-    def step_fused(sites=None, prm="prm"):
-        """The headline step: one spax_masked_gemv per token and site (mask outputs written)."""
+    def step_fused(sites=None, prm="prm", xsrc=None, ydst=None):
+        """The headline step: one spax_masked_gemv per token and site (mask outputs written).
+        xsrc / ydst: other input / output buffers (the end-to-end run's second set)."""
+        xsrc = xs if xsrc is None else xsrc
         for t in range(n_tok):
             for name, d_out, d_in, _ in SEL:
                 if sites is not None and name not in sites:
                     continue
                 b = buf[name]
-                spax.spax_masked_gemv(packed[name][t % n_rep], xs[name][t], b[prm], b["y"][t],
+                y = b["y"] if ydst is None else ydst[name]
+                spax.spax_masked_gemv(packed[name][t % n_rep], xsrc[name][t], b[prm], y[t],
                                       b["status"], b["ws"], tier=b["tier"][t],
                                       full_idx=b["fidx"][t], approx_idx=b["aidx"][t],
                                       counts=b["counts"][t], desc=b["desc"][t % n_rep])
@@ -362,6 +365,11 @@ def run_gpu(args, rank, world, local):
         return g
 
     graphs["fused"] = capture(step_fused)
+    # the end-to-end run's second buffer set: step i uses set i % 2, so the copies of one step
+    # overlap the compute of its neighbours
+    xs_b = {n: xs[n].clone() for n in xs}
+    y_b = {n: torch.empty_like(buf[n]["y"]) for n in xs}
+    graphs["fused_b"] = capture(step_fused, xsrc=xs_b, ydst=y_b)
     graphs["fused_unguessed"] = capture(step_fused, prm="prm_unguessed")
     graphs["fused_missed"] = capture(step_fused, prm="prm_missed")
     graphs["tiered"] = capture(step_tiered)
@@ -393,38 +401,65 @@ def run_gpu(args, rank, world, local):
                 time_graph(graphs["mask_" + name], args.steps, args.warmup, stream))
             res["dense_" + name] = max_over_ranks(
                 time_graph(graphs["dense_" + name], args.steps, args.warmup, stream))
-        # end to end: host inputs in, host outputs out, through the same C-ABI calls
+        # end to end: every step copies its inputs in from pinned host memory and its outputs
+        # back, through the same C-ABI calls. Two buffer sets, a copy-in and a copy-out stream:
+        # step i's copies overlap the compute of steps i - 1 and i + 1 (events keep each set's
+        # copy-in after the compute two steps back, and its compute after that step's copy-out).
         xin = {n: xs[n].cpu().pin_memory() for n in xs}
         yout = {n: torch.empty(buf[n]["y"].shape, dtype=torch.float32).pin_memory() for n in xs}
         h2d = sum(v.numel() * 4 for v in xin.values())
         d2h = sum(v.numel() * 4 for v in yout.values())
+        sets = [(xs, {n: buf[n]["y"] for n in xs}, graphs["fused"]), (xs_b, y_b, graphs["fused_b"])]
+        s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        ev_in = [torch.cuda.Event(), torch.cuda.Event()]
+        ev_comp = [torch.cuda.Event(), torch.cuda.Event()]
+        ev_out = [torch.cuda.Event(), torch.cuda.Event()]
 
-        def e2e_once():
-            for n in xs:
-                xs[n].copy_(xin[n], non_blocking=True)
-            graphs["fused"].replay()
-            for n in xs:
-                yout[n].copy_(buf[n]["y"], non_blocking=True)
+        def e2e_run(n_steps, start=None):
+            if start is not None:
+                s_in.wait_event(start)
+                s_out.wait_event(start)
+            for i in range(n_steps):
+                k = i % 2
+                xd, yd, g = sets[k]
+                with torch.cuda.stream(s_in):
+                    if i >= 2:
+                        s_in.wait_event(ev_comp[k])
+                    for n in xs:
+                        xd[n].copy_(xin[n], non_blocking=True)
+                    ev_in[k].record(s_in)
+                with torch.cuda.stream(stream):
+                    stream.wait_event(ev_in[k])
+                    if i >= 2:
+                        stream.wait_event(ev_out[k])
+                    g.replay()
+                    ev_comp[k].record(stream)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(ev_comp[k])
+                    for n in xs:
+                        yout[n].copy_(yd[n], non_blocking=True)
+                    ev_out[k].record(s_out)
+            for k in range(min(2, n_steps)):
+                stream.wait_event(ev_out[k])
 
-        with torch.cuda.stream(stream):
-            for _ in range(args.warmup):
-                e2e_once()
-            torch.cuda.synchronize()
-            barrier()
-            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            s0.record(stream)
-            for _ in range(args.steps):
-                e2e_once()
-            s1.record(stream)
-            torch.cuda.synchronize()
-            barrier()
+        e2e_run(max(2, args.warmup))
+        torch.cuda.synchronize()
+        barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        e2e_run(args.steps, start=s0)
+        s1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
         res["e2e"] = max_over_ranks(s0.elapsed_time(s1) / args.steps)
     for name, *_ in SEL:
         st = int(buf[name]["status"].item())
         if st != 0:
             raise RuntimeError(f"device status {st} after timing at site {name}")
-        if not torch.isfinite(buf[name]["y"]).all():
+        if not torch.isfinite(buf[name]["y"]).all() or not torch.isfinite(y_b[name]).all():
             raise RuntimeError(f"non-finite output at site {name}")
+        if not torch.equal(buf[name]["y"], y_b[name]):  # same inputs, same launches
+            raise RuntimeError(f"the two end-to-end buffer sets disagree at site {name}")
 
     launches_per_step = n_tok * len(SEL)
     sites = {}
@@ -904,7 +939,10 @@ def main():
                          "traffic": traffic,
                          "algorithmic_bytes_per_launch": round(tot_bytes / args.tokens / len(sites))},
             "e2e": {"value": round(e2e, 3), "unit": "us/token/layer", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
+                    "d2h_bytes_per_step": d2h,
+                    "note": "every step copies its inputs in from pinned host memory and its "
+                            "outputs back; two buffer sets and separate copy streams overlap a "
+                            "step's copies with its neighbours' compute"},
             "gpu_launches": lps * args.steps,
             "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
         }
