@@ -250,3 +250,33 @@ def test_masked_gemv_guess_bitexact(d_out, d_in):
         for o in outs[1:]:
             for a, b in zip(outs[0], o):
                 assert np.array_equal(a, b), f"token {tok}: guessed result differs"
+
+
+@pytest.mark.parametrize("d", [4096, 11008])
+def test_guess_miss_stress(d):
+    """Many tokens whose guesses all miss (twice and half the true keys, both boundaries or one):
+    the windowed pass gives way to the full selection in the same launch, which must start from a
+    clean histogram every time. Mask and one-launch masked GEMV against the oracle, bit for bit."""
+    m = Mask(d)
+    d_out = 1024
+    W = synth.weight(d_out, d, 4, 6, device="cuda")
+    pm = spax.alloc_packed(d_out, d, spax.FULL_BF16)
+    spax.spax_pack_weights(W, spax.FULL_BF16, pm)
+    ws = spax.alloc_workspace(spax.OP_TIERED_GEMV, d_out, d)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kf, ka = int(0.3 * d + 0.5), int(0.3 * d + 0.5)
+    for tok in range(24):
+        x = _laplace(d, 500 + tok)
+        f = (2.0, 0.5, 1.0)[tok % 3]
+        g = (1.0, 2.0, 0.5)[tok % 3]
+        tf, ts = kth_key(x, kf) * f, kth_key(x, kf + ka) * g
+        assert "miss" in (guess_path(x, kf, tf), guess_path(x, kf + ka, ts))
+        m.check(x, kf, ka, tf, ts, f"token {tok}")
+        prm = spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka, t_full=tf, t_skip=ts)
+        tier = torch.empty(d, dtype=torch.uint8, device="cuda")
+        y = torch.empty(d_out, device="cuda")
+        spax.spax_masked_gemv(pm, torch.from_numpy(x).cuda(), prm, y, st, ws, tier=tier)
+        torch.cuda.synchronize()
+        assert st.item() == 0
+        _, t_o, _, _, _ = oracle.tiers(x, oracle.MODE_TOPK, k_full=kf, k_approx=ka)
+        assert np.array_equal(tier.cpu().numpy(), t_o), f"masked GEMV token {tok}"

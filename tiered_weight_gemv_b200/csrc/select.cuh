@@ -598,9 +598,10 @@ __device__ __forceinline__ int select_topk_guessed(const spax_mask_params& prm, 
   __syncthreads();
   if (S.hint[4] >= 0x7F800000u) return 2;  // Inf / NaN among the keys
   const uint32_t A0 = S.hint[0], A1 = S.hint[2];
-  auto unwind = [&]() {  // a miss: the unhinted selection needs S.hist zero
+  auto unwind = [&]() {  // a miss (block-uniform): the unhinted selection needs S.hist zero
     for (int i = 4 * tid; i < kSelBins; i += 4 * kSelThreads)
       *reinterpret_cast<uint4*>(&S.hist[i]) = make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();  // pass 1 adds into S.hist at once: every bin is zero before any thread does
     return 0;
   };
   // rank K lies in the window iff the scan from the top finds it before the window's bottom
