@@ -580,14 +580,30 @@ def run_extras(args, dev):
                            ws=spax.alloc_workspace(spax.OP_TIERED_GEMV, d_out, d_in, device=dev),
                            dws=spax.alloc_workspace(spax.OP_DENSE_GEMV, d_out, d_in, device=dev))
         layer[name]["Xh"] = layer[name]["X"].to(torch.bfloat16)
+        # calibration tokens of the site's own distribution, never timed (the boundary guesses)
+        layer[name]["cal"] = synth.laplace((N_CAL, d_in), 8, tid + 10, device=dev)
+        layer[name]["cal_ws"] = torch.empty(spax.spax_workspace_bytes(spax.OP_CALIBRATE, 0, d_in),
+                                            dtype=torch.uint8, device=dev)
     torch.cuda.synchronize()
+    t_cal = torch.empty(2, device=dev)
+    st_cal = torch.zeros(1, dtype=torch.int32, device=dev)
     points = []
     for f, a in LLAMA3_POINTS:
-        prms = {name: spax.mask_params(spax.MASK_TOPK, k_full=int(math.floor(f * d_in + 0.5)),
-                                       k_approx=int(math.floor(a * d_in + 0.5)))
-                for name, _, d_in, _ in LLAMA3_SITES}
+        prms, prms0 = {}, {}
+        for name, _, d_in, _ in LLAMA3_SITES:
+            kf, ka = int(math.floor(f * d_in + 0.5)), int(math.floor(a * d_in + 0.5))
+            L = layer[name]
+            spax.spax_calibrate_thresholds(L["cal"], round((d_in - kf - ka) * 10000 / d_in),
+                                           round((d_in - kf) * 10000 / d_in), t_cal, st_cal,
+                                           L["cal_ws"])
+            t_skip, t_full = (float(v) for v in t_cal.cpu())
+            prms[name] = spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka, t_skip=t_skip,
+                                          t_full=t_full)
+            prms0[name] = spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka)
+        if int(st_cal.item()) != 0:
+            raise RuntimeError(f"calibration status {int(st_cal.item())} in the sweep")
 
-        def fn(prms=prms):
+        def fn(prms):
             for t in range(n_tok):
                 for name, *_ in LLAMA3_SITES:
                     L = layer[name]
@@ -595,10 +611,12 @@ def run_extras(args, dev):
                     spax.spax_masked_gemv(L["reps"][r], L["X"][t], prms[name], L["y"][t], L["st"],
                                           L["ws"], desc=L["descs"][r])
 
-        ms = timed(fn)
+        ms = timed(lambda: fn(prms))
+        ms0 = timed(lambda: fn(prms0))
         by = sum(fused_bytes(d_out, d_in, prms[n].k_full, prms[n].k_approx)
                  for n, d_out, d_in, _ in LLAMA3_SITES)
         points.append({"full": f, "approx": a, "us_per_token_layer": round(ms * 1000 / n_tok, 3),
+                       "unguessed_us_per_token_layer": round(ms0 * 1000 / n_tok, 3),
                        "bytes_per_token_layer": by,
                        "GBps": round(by * n_tok / (ms * 1e-3) / 1e9, 1)})
     for name, *_ in LLAMA3_SITES:
@@ -627,6 +645,10 @@ def run_extras(args, dev):
         "tokens": n_tok, "replicas": n_rep, "points": points,
         "fit_time_vs_bytes": fit_c0_bw([(p["bytes_per_token_layer"], p["us_per_token_layer"])
                                         for p in points]),
+        "unguessed_fit_time_vs_bytes": fit_c0_bw([(p["bytes_per_token_layer"],
+                                                   p["unguessed_us_per_token_layer"]) for p in points]),
+        "guess_note": "the TopK parameters carry |x| quantiles calibrated on 16 separate tokens per "
+                      "site and point; unguessed_* is the same launch sequence without them",
         "dense_us_per_token_layer": round(ms_dense * 1000 / n_tok, 3),
         "dense_GBps": round(dense_bytes * n_tok / (ms_dense * 1e-3) / 1e9, 1),
         "torch_mv_bf16_us_per_token_layer": round(ms_mv * 1000 / n_tok, 3),
