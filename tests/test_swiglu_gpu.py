@@ -79,9 +79,16 @@ def test_swiglu_input_matches_oracle(fmt, d_out, d_in):
     rows = np.unique(np.concatenate([np.arange(0, d_out, 41), np.arange(d_out - 3, d_out)]))
     gu = (2.0 * synth.laplace((2 * d_in,), 11, 1001 + d_out % 89, device="cuda")).contiguous()
     kf, ka = (3 * d_in + 5) // 10, (3 * d_in + 5) // 10
+    # a TopK guess of the boundary keys: quantiles of |silu(g) * u| (computed here in fp64)
+    xg = np.abs(oracle.swiglu(gu[:d_in].cpu().double().numpy(), gu[d_in:].cpu().double().numpy()))
+    gs, gf = np.quantile(xg, [1 - (kf + ka) / d_in, 1 - kf / d_in])
+    ys = []
     for prm in [spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka),
+                spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka, t_skip=float(gs),
+                                 t_full=float(gf)),
                 spax.mask_params(spax.MASK_THRESHOLD, t_skip=0.2, t_full=0.9)]:
-        _check(gm, pools, gu, prm, rows)
+        ys.append(_check(gm, pools, gu, prm, rows)["y"])
+    assert np.array_equal(ys[0], ys[1]), "the guess changed y"
     # an offset view of a larger buffer: g, u and x_out not 16-byte aligned (scalar path)
     big = torch.zeros(2 * d_in + 1, device="cuda")
     big[1:] = gu

@@ -72,9 +72,15 @@ def test_wina_masked_gemv_matches_oracle(fmt, d_out, d_in):
     rows = np.unique(np.concatenate([np.arange(0, d_out, 37), np.arange(d_out - 3, d_out)]))
     kf, ka = (3 * d_in + 5) // 10, (3 * d_in + 5) // 10
     ts, tf = np.quantile(score, [0.4, 0.7]).astype(np.float32)
+    # a TopK guess of the boundary keys is on the score, like every other key of this rule
+    gs, gf = np.quantile(score, [1 - (kf + ka) / d_in, 1 - kf / d_in])
+    ys = []
     for prm in [spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka),
+                spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka, t_skip=float(gs),
+                                 t_full=float(gf)),
                 spax.mask_params(spax.MASK_THRESHOLD, t_skip=float(ts), t_full=float(tf))]:
         r = _run(gm, x, norms, prm)
+        ys.append(r["y"])
         assert r["status"][0] == 0
         op = oracle_params(prm)
         st, t_o, f_o, a_o, c_o = oracle.tiers(score, op.pop("mode"), **op)
@@ -82,6 +88,7 @@ def test_wina_masked_gemv_matches_oracle(fmt, d_out, d_in):
         assert np.array_equal(r["fidx"][: c_o[0]], f_o) and np.array_equal(r["aidx"][: c_o[1]], a_o)
         y_ref = oracle.tiered_gemv(*pools, fmt, d_out, d_in, xh, t_o, rows=rows)
         check_y(r["y"][rows], y_ref)
+    assert np.array_equal(ys[0], ys[1]), "the guess changed y"
 
 
 def test_wina_with_equal_norms_is_the_magnitude_rule():
