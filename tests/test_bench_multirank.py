@@ -69,8 +69,8 @@ def test_two_gloo_ranks(tmp_path):
     lines = [ln for ln in (tmp_path / "out0.txt").read_text().splitlines() if ln.strip()]
     assert len(lines) == 1
     line = json.loads(lines[0])
-    base = json.load(open(os.path.join(ROOT, "BASELINE.json")))
-    assert line["metric"] == base["metric"]
+    import bench
+    assert line["metric"] == bench.METRIC
     assert line["impl"] == "reference" and line["n_gpus"] == world
     assert line["higher_is_better"] is False and line["steps"] == 2 and line["warmup"] == 3
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
