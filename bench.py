@@ -367,8 +367,9 @@ def run_gpu(args, rank, world, local):
     graphs["fused"] = capture(step_fused)
     # the end-to-end run's second buffer set: step i uses set i % 2, so the copies of one step
     # overlap the compute of its neighbours
-    xs_b = {n: xs[n].clone() for n in xs}
-    y_b = {n: torch.empty_like(buf[n]["y"]) for n in xs}
+    names = [s[0] for s in SEL]  # the sites this run executes
+    xs_b = {n: xs[n].clone() for n in names}
+    y_b = {n: torch.empty_like(buf[n]["y"]) for n in names}
     graphs["fused_b"] = capture(step_fused, xsrc=xs_b, ydst=y_b)
     graphs["fused_unguessed"] = capture(step_fused, prm="prm_unguessed")
     graphs["fused_missed"] = capture(step_fused, prm="prm_missed")
@@ -405,11 +406,12 @@ def run_gpu(args, rank, world, local):
         # back, through the same C-ABI calls. Two buffer sets, a copy-in and a copy-out stream:
         # step i's copies overlap the compute of steps i - 1 and i + 1 (events keep each set's
         # copy-in after the compute two steps back, and its compute after that step's copy-out).
-        xin = {n: xs[n].cpu().pin_memory() for n in xs}
-        yout = {n: torch.empty(buf[n]["y"].shape, dtype=torch.float32).pin_memory() for n in xs}
+        xin = {n: xs[n].cpu().pin_memory() for n in names}
+        yout = {n: torch.empty(buf[n]["y"].shape, dtype=torch.float32).pin_memory() for n in names}
         h2d = sum(v.numel() * 4 for v in xin.values())
         d2h = sum(v.numel() * 4 for v in yout.values())
-        sets = [(xs, {n: buf[n]["y"] for n in xs}, graphs["fused"]), (xs_b, y_b, graphs["fused_b"])]
+        sets = [(xs, {n: buf[n]["y"] for n in names}, graphs["fused"]),
+                (xs_b, y_b, graphs["fused_b"])]
         s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
         ev_in = [torch.cuda.Event(), torch.cuda.Event()]
         ev_comp = [torch.cuda.Event(), torch.cuda.Event()]
@@ -425,7 +427,7 @@ def run_gpu(args, rank, world, local):
                 with torch.cuda.stream(s_in):
                     if i >= 2:
                         s_in.wait_event(ev_comp[k])
-                    for n in xs:
+                    for n in names:
                         xd[n].copy_(xin[n], non_blocking=True)
                     ev_in[k].record(s_in)
                 with torch.cuda.stream(stream):
@@ -436,7 +438,7 @@ def run_gpu(args, rank, world, local):
                     ev_comp[k].record(stream)
                 with torch.cuda.stream(s_out):
                     s_out.wait_event(ev_comp[k])
-                    for n in xs:
+                    for n in names:
                         yout[n].copy_(yd[n], non_blocking=True)
                     ev_out[k].record(s_out)
             for k in range(min(2, n_steps)):
