@@ -207,11 +207,14 @@ spax_status spax_build_mask(const float* d_x, int d_in, const spax_mask_params* 
  * Accumulation is fp32, split over CTAs, then reduced in a fixed order (bit-reproducible for a
  * given GPU model and shape). Workspace: spax_workspace_bytes(SPAX_OP_TIERED_GEMV, d_out, d_in)
  * bytes, ZEROED BEFORE FIRST USE: it holds the split-K partial sums as flagged words that every
- * completed call leaves at zero (zero it again after a device error). The CTAs that split a row
- * tile wait for one another's partial sums (a wait bounded at 1 s, then SPAX_ERR_TIMEOUT): the
- * launch is one wave of at most one CTA per SM and expects its whole grid to be resident at
- * once. Counts outside [0, d_in] or an index outside [0, d_in) set *d_status = SPAX_ERR_INDEX;
- * such a column contributes zero. Calls that share a workspace must not run concurrently.
+ * completed call leaves at zero (zero it again after a device error). Counts outside [0, d_in]
+ * or an index outside [0, d_in) set *d_status = SPAX_ERR_INDEX; such a column contributes zero.
+ * Calls that share a workspace must not run concurrently.
+ * Residency: the CTAs that split a row tile wait for one another's partial sums (a wait bounded
+ * at 1 s, then SPAX_ERR_TIMEOUT and an unspecified y). The launch is one wave of at most one CTA
+ * per SM and needs its whole grid resident at once, which holds when the call has the GPU's SMs
+ * to itself: no kernel of another stream or process holding SMs while it runs, and no context
+ * limited to a subset of the SMs (MPS thread limits, green contexts).
  */
 spax_status spax_tiered_gemv(const spax_packed* h_W, const float* d_x, const int32_t* d_full_idx,
                              const int32_t* d_approx_idx, const int32_t* d_counts, float* d_y,
@@ -272,6 +275,22 @@ spax_status spax_masked_gemv_swiglu(const spax_packed* h_W, const float* d_gu,
                                     size_t ws_bytes, void* stream);
 
 /*
+ * spax_test_tiered_gemv_timeout — failure-detection test hook, not a computation. It launches
+ * the list-driven GEMV of spax_tiered_gemv with the last column split of every row tile left
+ * out, so the CTAs that wait for that split's partial sums give up after wait_limit_ns and set
+ * *d_status = SPAX_ERR_TIMEOUT, leaving the context usable. Afterwards y is unspecified and the
+ * scratch holds flagged words: zero the workspace (or call spax_fixed_scratch_reset) before the
+ * next GEMV. d_ws NULL selects the fixed scratch array of spax_tiered_gemv_fixed_scratch.
+ * Requires a shape whose plan has at least 2 splits (SPAX_ERR_SHAPE otherwise) and
+ * 1e6 <= wait_limit_ns <= 2e9. Other arguments as spax_tiered_gemv.
+ */
+spax_status spax_test_tiered_gemv_timeout(const spax_packed* h_W, const float* d_x,
+                                          const int32_t* d_full_idx, const int32_t* d_approx_idx,
+                                          const int32_t* d_counts, float* d_y, int32_t* d_status,
+                                          void* d_ws, size_t ws_bytes, uint64_t wait_limit_ns,
+                                          void* stream);
+
+/*
  * spax_dense_gemv — the same-GPU dense baseline: y = W x over every column, read from the
  * bf16 full pool (W^T [d_in][d_out]) with the same kernel family as spax_tiered_gemv.
  * Source: eigenradar commentary (comparisons use dense decoding in the same weight format).
@@ -287,21 +306,34 @@ spax_status spax_dense_gemv(const void* d_Wt, const float* d_x, float* d_y, int 
  * memory where they call it: its split-K scratch is a fixed array compiled into the library
  * (spax_fixed_scratch_bytes() = 4 MiB per device), so the call allocates nothing. The pages
  * have no counterpart of this entry point; it is an interface convenience.
- * - The first call on each device (with that device current) looks up the array's device
- *   address and caches it; make that first call before any stream capture on that device.
+ * - The first call in each device's context (with that device current) looks up the array's
+ *   device address and caches it; make that first call before any stream capture on that
+ *   device. The cache is keyed on the context's process-unique id, so after a cudaDeviceReset
+ *   the next call looks the address up again (the new context's array starts at zero).
  * - Shapes whose split plan needs more partial sums than the array holds are rejected with
  *   SPAX_ERR_WORKSPACE before anything is launched (none on a 148-SM GPU: a plan with splits
  *   needs at most S * d_out * 8 <= 148 * 2048 * 8 bytes, and one without needs none).
- * - The array starts at zero when the library loads and every completed call leaves it at zero;
- *   nothing for the caller to initialise.
+ * - The array starts at zero when the library loads and every completed call leaves it at zero.
+ *   A call that ends in a device error (SPAX_ERR_TIMEOUT, or a sticky CUDA error) may leave
+ *   flagged partial sums in it, which a later call would take for its own: after any such error,
+ *   call spax_fixed_scratch_reset before the next fixed-scratch call.
  * - There is ONE array per device for the whole process: calls on the same device that can
  *   overlap (other streams, other threads, concurrent graph branches) race on it and give
  *   wrong results. Serialise them.
+ * - Like spax_tiered_gemv, the launch needs its whole grid (one CTA per SM) resident at once:
+ *   see the residency note there.
  */
 spax_status spax_tiered_gemv_fixed_scratch(const spax_packed* h_W, const float* d_x,
                                            const int32_t* d_full_idx, const int32_t* d_approx_idx,
                                            const int32_t* d_counts, float* d_y, int32_t* d_status,
                                            void* stream);
+
+/*
+ * spax_fixed_scratch_reset — zero the current device's fixed scratch array (one
+ * cudaMemsetAsync on `stream`; allocates nothing). Call it after a fixed-scratch call reported
+ * SPAX_ERR_TIMEOUT or any device error, ordered after that call and before the next one.
+ */
+spax_status spax_fixed_scratch_reset(void* stream);
 
 /* Size in bytes of the per-device scratch array spax_tiered_gemv_fixed_scratch uses. */
 size_t spax_fixed_scratch_bytes(void);

@@ -177,7 +177,8 @@ spax_status spax_gemv_plan(int op, int d_out, int d_in, int full_fmt, int32_t* s
 static spax_status gemv_common(const void* full, const void* approx, int full_fmt, const float* x,
                                const int32_t* fidx, const int32_t* aidx, const int32_t* counts,
                                float* y, int d_out, int d_in, int32_t* status, void* ws,
-                               size_t ws_bytes, void* stream, bool dense) {
+                               size_t ws_bytes, void* stream, bool dense,
+                               unsigned long long wait_ns = 0, int drop_splits = 0) {
   if (!full || !x || !y) return SPAX_ERR_ARG;
   if (!dense && (!approx || !fidx || !aidx || !counts)) return SPAX_ERR_ARG;
   if (full_fmt != SPAX_FULL_BF16 && full_fmt != SPAX_FULL_INT4_G128) return SPAX_ERR_ARG;
@@ -187,9 +188,12 @@ static spax_status gemv_common(const void* full, const void* approx, int full_fm
   if (sms < 1) return SPAX_ERR_CUDA;
   GemvPlan pl;
   if (!make_gemv_plan(d_out, d_in, full_fmt, sms, &pl)) return SPAX_ERR_SHAPE;
+  if (drop_splits && pl.S <= drop_splits) return SPAX_ERR_SHAPE;
   if (!ws || ws_bytes < pl.ws_bytes) return SPAX_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(ws) & 255u) return SPAX_ERR_ARG;
   GemvLaunch a;
+  a.wait_ns = wait_ns;
+  a.drop_splits = drop_splits;
   a.full = full;
   a.approx = approx;
   a.x = x;
@@ -283,6 +287,21 @@ spax_status spax_masked_gemv_swiglu(const spax_packed* W, const float* gu,
                                     void* stream) {
   return masked_gemv_common(W, gu, true, x_out, nullptr, p, y, tier, full_idx, approx_idx, counts,
                             status, ws, ws_bytes, stream);
+}
+
+spax_status spax_test_tiered_gemv_timeout(const spax_packed* W, const float* x,
+                                          const int32_t* full_idx, const int32_t* approx_idx,
+                                          const int32_t* counts, float* y, int32_t* status,
+                                          void* ws, size_t ws_bytes, uint64_t wait_limit_ns,
+                                          void* stream) {
+  if (!W) return SPAX_ERR_ARG;
+  if (wait_limit_ns < 1000000ull || wait_limit_ns > 2000000000ull) return SPAX_ERR_ARG;
+  if (!ws) {  // the fixed scratch array of spax_tiered_gemv_fixed_scratch
+    ws = fixed_scratch_current_device_ptr(&ws_bytes);
+    if (!ws) return SPAX_ERR_CUDA;
+  }
+  return gemv_common(W->d_full, W->d_approx, W->full_fmt, x, full_idx, approx_idx, counts, y,
+                     W->d_out, W->d_in, status, ws, ws_bytes, stream, false, wait_limit_ns, 1);
 }
 
 spax_status spax_dense_gemv(const void* Wt, const float* x, float* y, int d_out, int d_in,

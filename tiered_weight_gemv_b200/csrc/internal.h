@@ -32,6 +32,8 @@ struct GemvLaunch {
   void* ws;
   int d_out, d_in, full_fmt;
   bool dense;
+  unsigned long long wait_ns = 0;  // bound of the split-K wait (0: kWaitLimitNs)
+  int drop_splits = 0;  // failure-detection test only: launch the last drop_splits splits of no tile
 };
 cudaError_t launch_gemv(const GemvLaunch& a, const GemvPlan& plan, cudaStream_t stream);
 // The mask and the GEMV in one launch (every CTA computes the token's lists itself); the tier,
@@ -54,6 +56,10 @@ cudaError_t launch_pack(const void* W, int d_out, int d_in, int full_fmt, void* 
                         cudaStream_t stream);
 cudaError_t launch_column_norms(const void* W, int d_out, int d_in, float* norms,
                                 cudaStream_t stream);
+
+// The fixed scratch array of spax_tiered_gemv_fixed_scratch on the current device (nullptr if
+// its address could not be looked up); *bytes gets its size.
+uint8_t* fixed_scratch_current_device_ptr(size_t* bytes);
 
 size_t calibrate_ws_bytes();
 cudaError_t launch_calibrate(const float* X, long long M, long long idx_skip, long long idx_full,

@@ -24,24 +24,71 @@ constexpr size_t kFixedScratchBytes = size_t(4) << 20;  // 4 MiB per device
 
 static __device__ __align__(256) uint8_t g_fixed_scratch[kFixedScratchBytes];
 
-// Device address of g_fixed_scratch on the current device, looked up once per device (with that
-// device current) and cached; nullptr if the lookup failed.
+// Driver calls the address cache needs, resolved through the runtime (no link-time dependency on
+// the driver library): the current context and its process-unique id.
+using CtxGetCurrentFn = int (*)(void** ctx);                       // cuCtxGetCurrent
+using CtxGetIdFn = int (*)(void* ctx, unsigned long long* id);     // cuCtxGetId
+
+// Id of the context current on this thread; false when there is none (or the driver lacks the
+// call), in which case the caller looks the address up again on every call.
+static bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(f);
+    (void)cudaGetLastError();
+  });
+  if (!get_current || !get_id) return false;
+  void* ctx = nullptr;
+  if (get_current(&ctx) != 0 || !ctx) return false;
+  return get_id(ctx, id) == 0;
+}
+
+// Device address of g_fixed_scratch in the current device's context; nullptr if the lookup
+// failed. It is looked up (cudaGetSymbolAddress, with that device current) the first time a
+// device's context calls in, and again whenever that device's context has changed since (a
+// cudaDeviceReset makes a new context, whose copy of the library's module is a new array, zero
+// again). Contexts are told apart by their process-unique id, not by handle.
 static uint8_t* fixed_scratch_current_device() {
   constexpr int kMaxDevices = 64;
+  struct Entry {
+    unsigned long long ctx_id;
+    uint8_t* addr;
+  };
   static std::mutex mu;
-  static uint8_t* addr[kMaxDevices] = {};
+  static Entry cache[kMaxDevices] = {};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lk(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_fixed_scratch) != cudaSuccess) {
-      (void)cudaGetLastError();
-      return nullptr;
-    }
-    addr[dev] = static_cast<uint8_t*>(p);
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    (void)cudaGetLastError();
+    return nullptr;
   }
-  return addr[dev];
+  unsigned long long id = 0;
+  bool have_id = current_context_id(&id);
+  std::lock_guard<std::mutex> lk(mu);
+  if (have_id && cache[dev].addr && cache[dev].ctx_id == id) return cache[dev].addr;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_fixed_scratch) != cudaSuccess || !p) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  if (!have_id) have_id = current_context_id(&id);  // the lookup made the context current
+  cache[dev].addr = static_cast<uint8_t*>(p);
+  cache[dev].ctx_id = have_id ? id : 0;  // id 0 is never a context's: the next call looks again
+  return cache[dev].addr;
+}
+
+uint8_t* fixed_scratch_current_device_ptr(size_t* bytes) {
+  if (bytes) *bytes = kFixedScratchBytes;
+  return fixed_scratch_current_device();
 }
 
 }  // namespace spax
@@ -51,6 +98,17 @@ using namespace spax;
 extern "C" {
 
 size_t spax_fixed_scratch_bytes(void) { return kFixedScratchBytes; }
+
+spax_status spax_fixed_scratch_reset(void* stream) {
+  uint8_t* scratch = fixed_scratch_current_device();
+  if (!scratch) return SPAX_ERR_CUDA;
+  if (cudaMemsetAsync(scratch, 0, kFixedScratchBytes, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess) {
+    (void)cudaGetLastError();
+    return SPAX_ERR_CUDA;
+  }
+  return SPAX_OK;
+}
 
 spax_status spax_tiered_gemv_fixed_scratch(const spax_packed* W, const float* x,
                                            const int32_t* full_idx, const int32_t* approx_idx,

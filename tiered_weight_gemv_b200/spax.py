@@ -69,6 +69,9 @@ _SIGS = {
     "spax_tiered_gemv_fixed_scratch": ([ctypes.POINTER(spax_packed), _P, _P, _P, _P, _P, _P, _P],
                                        _I),
     "spax_fixed_scratch_bytes": ([], _Z),
+    "spax_fixed_scratch_reset": ([_P], _I),
+    "spax_test_tiered_gemv_timeout": ([ctypes.POINTER(spax_packed), _P, _P, _P, _P, _P, _P, _P, _Z,
+                                      ctypes.c_uint64, _P], _I),
     "spax_workspace_bytes": ([_I, _I, _I], _Z),
     "spax_gemv_plan": ([_I, _I, _I, _I, _P, _P], _I),
     "spax_block_budgets": ([_P, _I, ctypes.c_double, ctypes.c_double, ctypes.c_double,
@@ -351,6 +354,29 @@ def spax_tiered_gemv_fixed_scratch(W: PackedMatrix, x: torch.Tensor, full_idx: t
 
 def spax_fixed_scratch_bytes() -> int:
     return int(_lib.spax_fixed_scratch_bytes())
+
+
+def spax_fixed_scratch_reset(stream=None) -> None:
+    """Zero the current device's fixed scratch array (after a fixed-scratch call reported a
+    device error such as ERR_TIMEOUT)."""
+    _check("spax_fixed_scratch_reset", _lib.spax_fixed_scratch_reset(_stream(stream)))
+
+
+def spax_test_tiered_gemv_timeout(W: PackedMatrix, x: torch.Tensor, full_idx: torch.Tensor,
+                                  approx_idx: torch.Tensor, counts: torch.Tensor, y: torch.Tensor,
+                                  status: torch.Tensor, ws=None, wait_limit_ns: int = 20_000_000,
+                                  stream=None) -> None:
+    """Failure-detection test hook: the list-driven GEMV with the last split of every row tile
+    left out, so its waits run out after wait_limit_ns and status becomes ERR_TIMEOUT. ws None
+    selects the fixed scratch array."""
+    d = W.desc()
+    _check("spax_test_tiered_gemv_timeout", _lib.spax_test_tiered_gemv_timeout(
+        ctypes.byref(d), _dev(x, torch.float32, "x"), _dev(full_idx, torch.int32, "full_idx"),
+        _dev(approx_idx, torch.int32, "approx_idx"), _dev(counts, torch.int32, "counts"),
+        _dev(y, torch.float32, "y"), _dev(status, torch.int32, "status"),
+        None if ws is None else _dev(ws, None, "ws"),
+        0 if ws is None else ws.numel() * ws.element_size(), int(wait_limit_ns),
+        _stream(stream)))
 
 
 def spax_dense_gemv(Wt: torch.Tensor, x: torch.Tensor, y: torch.Tensor, d_out: int, d_in: int,
