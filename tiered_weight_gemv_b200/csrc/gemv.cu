@@ -34,7 +34,7 @@
 //     that wait for one another are all resident; the wait is bounded (SPAX_ERR_TIMEOUT).
 #include "common.cuh"
 #include "internal.h"
-#include "select_fused.cuh"
+#include "select.cuh"
 
 namespace spax {
 
@@ -88,11 +88,6 @@ struct GemvParams {
   float* x_out;    // fused swiglu only: the token's x (lead CTA; may be null)
   const float* norms;  // fused only, may be null: rank by the WINA score |x_j| * norms[j]
   unsigned long long wait_ns;  // bound of the split-K wait
-  // fused (second form) only: this CTA's lists, the shared-memory area the selection shares with
-  // the combine area, and the split's division constant
-  int lcap;         // entries per local list
-  int alias_bytes;  // selection scratch + candidates | combine area
-  uint32_t smagic;  // split_magic(S)
 };
 
 // Code -> float: (word & (mask << p)) | bits(C) is the float C + code, exactly, when C = 2^(23-p)
@@ -150,11 +145,9 @@ __host__ __device__ inline size_t fused_select_bytes(int d) {
 // RGT: the row-tile factor fixed at compile time (1, 2, 4), or 0 for the launch's p.RG. The tiered
 // kernels take 0 (one image for every shape of a layer); the dense baseline, a pure stream that
 // gains from the constant, keeps one image per tile height.
-template <int RGT, int FMT, bool DENSE, int FV>
+template <int RGT, int FMT, bool DENSE, bool FUSED>
 __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const GemvParams p) {
   constexpr int U = kGemvU;
-  constexpr bool FUSED = FV != 0;  // the kernel runs the tier rule itself
-  constexpr bool V2 = FV == 2;     // ... in the form of select_fused.cuh
   const int RG = RGT > 0 ? RGT : p.RG, R = 512 * RG, CG = kGemvWarps / RG;
   const int kSlotFloats = RG * 576;  // combine slot of a column group: 36 floats per 32 rows
   static_assert(FMT == SPAX_FULL_BF16 || !DENSE, "the dense GEMV reads the bf16 pool");
@@ -163,17 +156,14 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
   int32_t* meta_col_a = reinterpret_cast<int32_t*>(smem);
   int32_t* meta_col_f = meta_col_a + kGemvMeta;
   uint16_t* list = reinterpret_cast<uint16_t*>(meta_col_f + kGemvMeta);  // FUSED: staged lists
-  // second fused form: [lf | la][x][selection scratch + candidates | combine][staging]
-  uint16_t* lf = reinterpret_cast<uint16_t*>(smem);
-  uint16_t* la = lf + p.lcap;
-  uint8_t* const lists_end = V2 ? smem + p.list_bytes : reinterpret_cast<uint8_t*>(list) + p.list_bytes;
-  float* red = reinterpret_cast<float*>(lists_end + p.keys_bytes);
+  float* red = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(list) + p.list_bytes +
+                                        p.keys_bytes);
   // fused, keys kept alive: x of every column for the product (null otherwise)
   const uint32_t* x_live = (FUSED && p.keys_bytes && !p.norms)
-                               ? reinterpret_cast<const uint32_t*>(lists_end)
+                               ? reinterpret_cast<const uint32_t*>(reinterpret_cast<uint8_t*>(list) +
+                                                                   p.list_bytes)
                                : nullptr;
   __shared__ int s_bad, s_last;
-  __shared__ alignas(16) uint32_t s_oscan[2 * kSelWarps];  // second form: the outputs' scans
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -186,8 +176,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
   const bool v0 = rb + 8 * lane < p.d_out;   // lane's first 8-row chunk is inside the matrix
   const bool v1 = rb + 256 + 8 * lane < p.d_out;
   // per-warp staging buffer: kBatch records, then their coefficients x*scale per 128-row group
-  uint8_t* stage = reinterpret_cast<uint8_t*>(red) + (V2 ? p.alias_bytes : kCombineFloats * 4) +
-                   warp * kStageWarpBytes;
+  uint8_t* stage = reinterpret_cast<uint8_t*>(red + kCombineFloats) + warp * kStageWarpBytes;
   const uint32_t stage_s = smem_u32(stage);
   const uint32_t coef_s = stage_s + kStageRecBytes;
 
@@ -197,45 +186,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
   }
   int Kf, Ka;
   uint32_t a0 = 0;  // FUSED: start of the approximate list in list[]
-  // second form: what the outputs need at the end
-  Boundary B2[2];
-  uint32_t n1v = 0, n2v = 0;
-  bool bad2 = false;
-  if constexpr (V2) {
-    // ---- the tier rule of this token (select_fused.cuh), computed by every CTA ----
-    SelectSmem& sel = *reinterpret_cast<SelectSmem*>(red);
-    uint16_t* cand = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(red) +
-                                                 (sizeof(SelectSmem) + 15) / 16 * 16);
-    uint32_t* keys = reinterpret_cast<uint32_t*>(lists_end);
-    select_zero(sel);
-    pdl_wait();
-    pdl_launch_dependents();
-    if (p.swiglu)
-      select_fetch_swiglu(p.x, p.d_in, keys, tile == 0 && split == 0 ? p.x_out : nullptr);
-    else if (p.norms)
-      select_fetch_scored(p.x, p.norms, p.d_in, keys);
-    else
-      select_fetch(p.x, p.d_in, keys);
-    Coarse C;
-    bad2 = fsel_coarse(p.prm, p.d_in, keys, sel, &n1v, &n2v, C);
-    uint32_t nCF = 0, nCA = 0, nC = 0;
-    if (!bad2)
-      fsel_certain(keys, p.d_in, C, (uint32_t)S, (uint32_t)split, p.smagic, lf, la,
-                   (uint32_t)p.lcap, cand, sel, &nCF, &nCA, &nC, &bad2);
-    if (bad2) {  // non-finite x: every tier 0, empty lists, y = 0
-      Kf = 0;
-      Ka = 0;
-      if (tid == 0) record_status(p.status, SPAX_ERR_NONFINITE);
-    } else {
-      fsel_resolve(keys, cand, nC, C, sel, B2);
-      uint32_t nBF, nBA;
-      fsel_boundary(keys, cand, nC, B2, nCF, nCA, (uint32_t)S, (uint32_t)split, p.smagic, lf, la,
-                    (uint32_t)p.lcap, sel, &nBF, &nBA);
-      Kf = (int)(nCF + nBF);
-      Ka = (int)(nCA + nBA);
-    }
-    __syncthreads();  // the selection's scratch is dead before the combine area reuses it
-  } else if constexpr (FUSED) {
+  if constexpr (FUSED) {
     // ---- the tier rule of this token, computed by every CTA (identical results) ----
     SelectSmem& sel = *reinterpret_cast<SelectSmem*>(red);
     uint32_t* keys = p.keys_bytes ? reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(list) +
@@ -353,7 +304,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
 
   // x of local position i of this split's approximate / full list: the fused kernel's stash
   // (first kGemvMeta positions), else x of the column
-  const int xs_lim = (FV == 1 && !p.norms && !p.keys_bytes) ? kGemvMeta : 0;  // stash positions
+  const int xs_lim = (FUSED && !p.norms && !p.keys_bytes) ? kGemvMeta : 0;  // stash positions
   auto xA = [&](int i, int col) -> float {
     if constexpr (FUSED) {
       if (x_live) return __uint_as_float(x_live[col]);
@@ -372,13 +323,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
   // Column of local position i of this split's approximate / full list (in the current chunk):
   // the fused kernel reads its staged lists directly, the list-driven one its metadata arrays.
   auto colA = [&](int i) -> int {
-    if constexpr (V2) return (int)la[i];
-    else if constexpr (FUSED) return (int)list[a0 + split + S * i];
+    if constexpr (FUSED) return (int)list[a0 + split + S * i];
     else return meta_col_a[i];
   };
   auto colF = [&](int i) -> int {
-    if constexpr (V2) return (int)lf[i];
-    else if constexpr (FUSED) return (int)list[split + S * i];
+    if constexpr (FUSED) return (int)list[split + S * i];
     else return meta_col_f[i];
   };
 
@@ -728,32 +677,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
     return v;
   };
 
-  // second form: the lead CTA writes the optional mask outputs in ascending order once its own
-  // partial rows are out (the others' arrive meanwhile)
-  auto write_outputs = [&]() {
-    if constexpr (V2) {
-      if (!(tile == 0 && split == 0)) return;
-      if (bad2) {
-        if (p.tier_out)
-          for (int j = tid; j < p.d_in; j += kGemvThreads) p.tier_out[j] = 0;
-      } else if (p.tier_out || p.fidx_out || p.aidx_out) {
-        fsel_write_outputs(reinterpret_cast<const uint32_t*>(lists_end), p.d_in, B2, s_oscan,
-                           p.tier_out, p.fidx_out, p.aidx_out);
-      }
-      if (tid == 0 && p.counts_out) {
-        const bool topk = p.prm.mode == SPAX_MASK_TOPK, thr = p.prm.mode == SPAX_MASK_THRESHOLD;
-        p.counts_out[0] = Kf;
-        p.counts_out[1] = Ka;
-        p.counts_out[2] = (bad2 || topk) ? 0 : (thr ? p.d_in - Kf - Ka : (int32_t)n1v);
-        p.counts_out[3] = (bad2 || topk) ? 0 : (thr ? p.d_in - Kf : (int32_t)n2v);
-      }
-    }
-  };
-
   if (S == 1) {  // no split: the tile's rows are final
     for (int i = tid; i < rows_here / 4; i += kGemvThreads)
       reinterpret_cast<float4*>(p.y + r0)[i] = combined_rows(i);
-    write_outputs();
     return;
   }
 
@@ -765,7 +691,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
   // every completed call leaves the partial area at zero.
   unsigned long long* part = p.part + (size_t)split * p.d_out + r0;
   for (int i = tid; i < rows_here / 4; i += kGemvThreads) st_ll4(part + 4 * i, combined_rows(i));
-  write_outputs();
   const int n4 = rows_here / 4;
   const int c4 = (n4 + S - 1) / S;
   const int g_lo = min(n4, split * c4), ng = min(n4, g_lo + c4) - g_lo;
@@ -843,24 +768,24 @@ bool make_gemv_plan(int d_out, int d_in, int full_fmt, int sm_count, GemvPlan* p
   return true;
 }
 
-template <int RGT, int FMT, bool DENSE, int FV>
+template <int RGT, int FMT, bool DENSE, bool FUSED>
 static cudaError_t launch_one(const GemvParams& gp, const GemvPlan& pl, size_t smem,
                               cudaStream_t stream) {
-  auto kern = tiered_gemv_kernel<RGT, FMT, DENSE, FV>;
+  auto kern = tiered_gemv_kernel<RGT, FMT, DENSE, FUSED>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), (int)smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(pl.T, pl.S), dim3(kGemvThreads), smem, stream, gp);
 }
 
-template <int FMT, bool DENSE, int FV>
+template <int FMT, bool DENSE, bool FUSED>
 static cudaError_t launch_r(const GemvParams& gp, const GemvPlan& pl, size_t smem,
                             cudaStream_t stream) {
   if constexpr (DENSE) {
-    if (pl.R == 512) return launch_one<1, FMT, DENSE, FV>(gp, pl, smem, stream);
-    if (pl.R == 1024) return launch_one<2, FMT, DENSE, FV>(gp, pl, smem, stream);
-    return launch_one<4, FMT, DENSE, FV>(gp, pl, smem, stream);
+    if (pl.R == 512) return launch_one<1, FMT, DENSE, FUSED>(gp, pl, smem, stream);
+    if (pl.R == 1024) return launch_one<2, FMT, DENSE, FUSED>(gp, pl, smem, stream);
+    return launch_one<4, FMT, DENSE, FUSED>(gp, pl, smem, stream);
   } else {
-    return launch_one<0, FMT, DENSE, FV>(gp, pl, smem, stream);
+    return launch_one<0, FMT, DENSE, FUSED>(gp, pl, smem, stream);
   }
 }
 
@@ -885,30 +810,7 @@ static size_t masked_gemv_layout(int d_in, size_t* keys_bytes) {
   return meta + select_list_bytes(d_in) + (gemv > sel ? gemv : sel);
 }
 
-// Shared memory of the second fused form (select_fused.cuh): [lf | la][x][selection scratch and
-// candidates, later the combine area][staging]. The local lists hold this split's positions of
-// both lists (at most ceil(d_in / S) + 1 each; lcap leaves room). Returns 0 when it does not fit
-// one CTA, in which case the first form serves the shape.
-struct Layout2 {
-  size_t list_bytes, keys_bytes, alias_bytes, total;
-  int lcap;
-};
-static Layout2 masked_gemv_layout2(const GemvPlan& pl, int d_in) {
-  Layout2 L;
-  L.lcap = (d_in + pl.S - 1) / pl.S + 8;
-  L.list_bytes = (size_t(2) * L.lcap * 2 + 15) / 16 * 16;
-  L.keys_bytes = select_keys_bytes(d_in);
-  const size_t sel = (sizeof(SelectSmem) + 15) / 16 * 16 + (size_t(2) * d_in + 15) / 16 * 16;
-  const size_t comb = size_t(kCombineFloats) * 4;
-  L.alias_bytes = sel > comb ? sel : comb;
-  L.total = L.list_bytes + L.keys_bytes + L.alias_bytes + size_t(kGemvWarps) * kStageWarpBytes;
-  if (L.total > kMaskedGemvSmemLimit) L.total = 0;
-  return L;
-}
-
-size_t masked_gemv_smem_bytes(const GemvPlan& pl, int d_in) {
-  const Layout2 L = masked_gemv_layout2(pl, d_in);
-  if (L.total) return L.total;
+size_t masked_gemv_smem_bytes(const GemvPlan& /*pl: every tile height takes the same*/, int d_in) {
   size_t kb;
   return masked_gemv_layout(d_in, &kb);
 }
@@ -944,9 +846,9 @@ cudaError_t launch_gemv(const GemvLaunch& a, const GemvPlan& pl, cudaStream_t st
   GemvPlan grid = pl;  // the launched grid: every split, or (a failure-detection test) fewer
   grid.S = pl.S - a.drop_splits;
   if (grid.S < 1) return cudaErrorInvalidValue;
-  if (a.dense) return launch_r<SPAX_FULL_BF16, true, 0>(gp, grid, smem, stream);
-  if (a.full_fmt == SPAX_FULL_BF16) return launch_r<SPAX_FULL_BF16, false, 0>(gp, grid, smem, stream);
-  return launch_r<SPAX_FULL_INT4_G128, false, 0>(gp, grid, smem, stream);
+  if (a.dense) return launch_r<SPAX_FULL_BF16, true, false>(gp, grid, smem, stream);
+  if (a.full_fmt == SPAX_FULL_BF16) return launch_r<SPAX_FULL_BF16, false, false>(gp, grid, smem, stream);
+  return launch_r<SPAX_FULL_INT4_G128, false, false>(gp, grid, smem, stream);
 }
 
 cudaError_t launch_masked_gemv(const GemvLaunch& a, const spax_mask_params& prm, bool swiglu,
@@ -962,22 +864,12 @@ cudaError_t launch_masked_gemv(const GemvLaunch& a, const spax_mask_params& prm,
   gp.fidx_out = full_idx;
   gp.aidx_out = approx_idx;
   gp.counts_out = counts;
-  const Layout2 L = masked_gemv_layout2(pl, a.d_in);
-  if (L.total) {  // the second form
-    gp.list_bytes = (int)L.list_bytes;
-    gp.keys_bytes = (int)L.keys_bytes;
-    gp.alias_bytes = (int)L.alias_bytes;
-    gp.lcap = L.lcap;
-    gp.smagic = split_magic((uint32_t)pl.S);
-    if (a.full_fmt == SPAX_FULL_BF16) return launch_r<SPAX_FULL_BF16, false, 2>(gp, pl, L.total, stream);
-    return launch_r<SPAX_FULL_INT4_G128, false, 2>(gp, pl, L.total, stream);
-  }
   gp.list_bytes = (int)select_list_bytes(a.d_in);
   size_t kb;
   const size_t smem = masked_gemv_layout(a.d_in, &kb);
   gp.keys_bytes = (int)kb;
-  if (a.full_fmt == SPAX_FULL_BF16) return launch_r<SPAX_FULL_BF16, false, 1>(gp, pl, smem, stream);
-  return launch_r<SPAX_FULL_INT4_G128, false, 1>(gp, pl, smem, stream);
+  if (a.full_fmt == SPAX_FULL_BF16) return launch_r<SPAX_FULL_BF16, false, true>(gp, pl, smem, stream);
+  return launch_r<SPAX_FULL_INT4_G128, false, true>(gp, pl, smem, stream);
 }
 
 }  // namespace spax

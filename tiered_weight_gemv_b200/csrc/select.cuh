@@ -60,7 +60,6 @@ struct SelectSmem {
   uint32_t sel[2][4];    // per boundary: prefix / key, count above, count in the bin
   alignas(16) uint32_t wsum[kSelWarps];
   alignas(16) uint32_t wscan[kSelWarps];
-  alignas(16) uint32_t wscan2[2 * kSelWarps];  // two-word block scans (select_fused.cuh)
   uint32_t hint[8];           // guessed TopK: #keys above each window (0, 2), the largest key
                               // (4), the keys gathered from one bin per boundary (5, 6)
   uint32_t cand[2][kSelCand]; // guessed TopK: those gathered keys
