@@ -56,6 +56,11 @@ __device__ __forceinline__ uint32_t lds32(uint32_t a) {
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
   return v;
 }
+__device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+  return v;
+}
 
 // ---- packed fp32x2 FMA (sm_100): d = a * b + c, two lanes per instruction -----------------------
 struct f2 {
@@ -74,9 +79,11 @@ __device__ __forceinline__ f2 ffma2(f2 a, f2 b, f2 c) {
 }
 
 // bf16 pair in one 32-bit word -> the two fp32 values (exact: bf16 is the top half of fp32).
+// The low half moves up by a multiply, which the compiler may issue on the FMA pipe and so
+// leave the integer pipe to the decoding of the small formats.
 __device__ __forceinline__ f2 bf16x2_to_f2(uint32_t w) {
   f2 r;
-  r.x = __uint_as_float(w << 16);
+  r.x = __uint_as_float(w * 65536u);
   r.y = __uint_as_float(w & 0xFFFF0000u);
   return r;
 }

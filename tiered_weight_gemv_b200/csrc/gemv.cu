@@ -18,9 +18,9 @@
 //     CTA's share. Lane l owns rows 8l..8l+7 and 256+8l..256+8l+7 in all three formats, so bf16,
 //     int4 and 2-bit contributions land in the same 16 fp32 accumulators. Weights stream straight
 //     into registers with 16-byte loads marked evict-first, U bf16 columns in flight per warp;
-//     the small 2-bit records come by cp.async into a per-warp double buffer in shared memory,
-//     a batch of 16 columns sent one batch ahead (int4 records are staged synchronously). A
-//     warp's short last bf16 round is fetched into the idle second buffer with the first loads.
+//     the small 2-bit and int4 records come by cp.async into a per-warp double buffer in shared
+//     memory, each batch sent one batch ahead. A warp's short last bf16 round is fetched into
+//     the idle second buffer with the first loads.
 //     (Measured on B200: one-warp-issued 1-D bulk copies of 0.1-4 KB column segments are
 //     issue-bound at 0.5-3 TB/s; plain 16-byte loads from many warps reach 6.4-6.9 TB/s.)
 //   * 2-bit and int4 codes become floats with one LOP3 each: the code is masked into the
@@ -44,13 +44,14 @@ constexpr int kGemvMeta = 1024;  // metadata slots per list per chunk
 constexpr int kGemvU = 4;        // columns in flight per warp
 
 // Small records (2-bit: 144 B per column and 512 rows; int4: 272 B per column and 512 rows) are
-// fetched a batch of 16 at a time into a per-warp staging buffer with coalesced 16-byte loads,
-// so a warp keeps 2-4 KB in flight instead of a few bytes per lane.
+// fetched a batch at a time by cp.async into a per-warp double buffer (16-byte pieces), the next
+// batch in flight while the current one is decoded, so a warp keeps 2-4 KB in flight instead of a
+// few bytes per lane.
 constexpr int kBatch2 = 16;                // 2-bit columns per staged batch
-constexpr int kBatch4 = 16;                // int4 columns per staged batch
+constexpr int kBatch4 = 8;                 // int4 columns per staged batch (two in flight)
 constexpr int kStage2Bytes = 16 * 144;      // one batch of 2-bit records
 constexpr int kStageRecBytes = 2 * kStage2Bytes;  // two 2-bit batches (>= one int4 batch, 16 * 272)
-constexpr int kStageWarpBytes = kStageRecBytes + 16 * 16;  // + 4 coefficients per column
+constexpr int kStageWarpBytes = kStageRecBytes + 16 * 32;  // + 4 coefficient pairs per column
 
 // Row tile of R = 512 RG rows (RG = 1, 2 or 4, a launch parameter): warp (rg, cg) takes rows
 // [512 rg, 512 rg + 512) of the tile and every CG-th column of the CTA's share, CG = 16 / RG.
@@ -59,7 +60,8 @@ constexpr int kStageWarpBytes = kStageRecBytes + 16 * 16;  // + 4 coefficients p
 constexpr int kCombineFloats = kGemvWarps * 576;  // CG slots of (R / 32) * 36 floats, any RG
 constexpr size_t kGemvSmemBytes = size_t(2) * kGemvMeta * 4 + size_t(kCombineFloats) * 4 +
                                   size_t(kGemvWarps) * kStageWarpBytes;
-static_assert(kBatch4 * 272 <= kStageRecBytes && 2 * kBatch2 * 144 <= kStageRecBytes, "staging");
+constexpr int kStage4Bytes = kBatch4 * 272;  // one batch of int4 half-records
+static_assert(2 * kStage4Bytes <= kStageRecBytes && 2 * kBatch2 * 144 <= kStageRecBytes, "staging");
 
 struct GemvParams {
   const uint8_t* full;
@@ -331,58 +333,21 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
     else return meta_col_f[i];
   };
 
-  // Stage nb (<= kBatch2) 2-bit records of columns colA(cg + CG*(k0 + k)) and prepare
-  // their coefficients c[k][g] = x*scale_g (lane k), accumulating the group sums.
-  auto stage_approx = [&](int k0, int nb) {
-    __syncwarp();
-    constexpr int kChunks2 = (kBatch2 * 9 + 31) / 32;  // 16-byte chunks per lane
-    uint4 v[kChunks2];
-#pragma unroll
-    for (int t = 0; t < kChunks2; ++t) {
-      const int q = t * 32 + lane, k = q / 9, piece = q - 9 * k;
-      const int col = k < nb ? max(colA(cg + CG * (k0 + k)), 0) : 0;
-      v[t] = k < nb ? ld_stream128(p.approx + col * p.approx_col_stride + off_approx + 16 * piece)
-                    : make_uint4(0u, 0u, 0u, 0u);
-    }
-    float xk = 0.f;
-    if (lane < nb) {
-      const int i = cg + CG * (k0 + lane), col = colA(i);
-      xk = col >= 0 ? xA(i, col) : 0.f;  // an invalid column contributes zero
-    }
-#pragma unroll
-    for (int t = 0; t < kChunks2; ++t)
-      if (t * 32 + lane < kBatch2 * 9) reinterpret_cast<uint4*>(stage)[t * 32 + lane] = v[t];
-    __syncwarp();
-    if (lane < nb) {
-      const uint4 sm = lds128(stage_s + 144 * lane + 128);  // (scale | min << 16) per group
-      const uint32_t w[4] = {sm.x, sm.y, sm.z, sm.w};
-      float c[4];
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        c[g] = xk * __uint_as_float(w[g] << 16);
-        sA[g] += c[g];
-        bA[g] = fmaf(xk, __uint_as_float(w[g] & 0xFFFF0000u), bA[g]);
-      }
-      asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(coef_s + 16 * lane), "f"(c[0]),
-                   "f"(c[1]), "f"(c[2]), "f"(c[3]));
-    }
-    __syncwarp();
-  };
-
-  // 2-bit column k of the staged batch: 16 rows per word, row k at bits 2k. Rotations by 17 and
-  // 25 bring rows 0-3 and 4-7 of an 8-row group to mantissa bits 15, 17, 19, 21: values 256+q,
-  // 64+q, 16+q, 4+q.
+  // 2-bit column k of the staged batch: a lane's 8 rows in 16 bits, row i at bits 2i. Shifts left
+  // by 15 and 7 (multiplies, which the FMA pipe can take) bring rows 0-3 and 4-7 to mantissa bits
+  // 15, 17, 19, 21: values 256+q, 64+q, 16+q, 4+q. The coefficient comes as a ready pair.
   auto decode_approx = [&](int k, int buf = 0) {
     const uint32_t rec = stage_s + kStage2Bytes * buf + 144 * k;
-    const uint32_t q01 = lds32(rec + 2 * (lane & ~1)) >> (16 * (lane & 1));  // 2 bytes at 2*lane
-    const uint32_t q11 = lds32(rec + 64 + 2 * (lane & ~1)) >> (16 * (lane & 1));
-    const float c0 = __uint_as_float(lds32(coef_s + 16 * k + 4 * (lane / 16)));
-    const float c1 = __uint_as_float(lds32(coef_s + 16 * k + 4 * (2 + lane / 16)));
+    const uint32_t q01 = lds_u16(rec + 2 * lane);  // rows 8l .. 8l+7
+    const uint32_t q11 = lds_u16(rec + 64 + 2 * lane);  // rows 256+8l .. 256+8l+7
+    const uint2 p0 = lds64(coef_s + 32 * k + 8 * (lane / 16));
+    const uint2 p1 = lds64(coef_s + 32 * k + 8 * (2 + lane / 16));
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
       const uint32_t w = b ? q11 : q01;
-      const f2 c2 = b ? f2{c1, c1} : f2{c0, c0};
-      const uint32_t ra = __funnelshift_r(w, w, 17), rc = __funnelshift_r(w, w, 25);
+      const uint2 pc = b ? p1 : p0;
+      const f2 c2{__uint_as_float(pc.x), __uint_as_float(pc.y)};
+      const uint32_t ra = w * 32768u, rc = w * 128u;
       acc[4 * b + 0] = ffma2(f2{code_f(ra, 3u << 15, 0x43800000u), code_f(ra, 3u << 17, 0x42800000u)}, c2, acc[4 * b + 0]);
       acc[4 * b + 1] = ffma2(f2{code_f(ra, 3u << 19, 0x41800000u), code_f(ra, 3u << 21, 0x40800000u)}, c2, acc[4 * b + 1]);
       acc[4 * b + 2] = ffma2(f2{code_f(rc, 3u << 15, 0x43800000u), code_f(rc, 3u << 17, 0x42800000u)}, c2, acc[4 * b + 2]);
@@ -420,8 +385,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
         sA[g] += c[g];
         bA[g] = fmaf(xk, __uint_as_float(w[g] & 0xFFFF0000u), bA[g]);
       }
-      asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(coef_s + 16 * lane), "f"(c[0]),
-                   "f"(c[1]), "f"(c[2]), "f"(c[3]));
+      asm volatile("st.shared.v4.f32 [%0], {%1, %1, %2, %2};" ::"r"(coef_s + 32 * lane), "f"(c[0]),
+                   "f"(c[1]));
+      asm volatile("st.shared.v4.f32 [%0], {%1, %1, %2, %2};" ::"r"(coef_s + 32 * lane + 16),
+                   "f"(c[2]), "f"(c[3]));
     }
     __syncwarp();
   };
@@ -552,41 +519,40 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
         }
       }
     } else {
+      // the 2-bit tier: batches double-buffered by cp.async, as in the bf16 path
+      if (nAw > 0) stage_issue(0, min(kBatch2, nAw), 0);
       for (int ka = 0; ka < nAw; ka += kBatch2) {
-        const int nb = min(kBatch2, nAw - ka);
-        stage_approx(ka, nb);
+        const int nb = min(kBatch2, nAw - ka), buf = (ka / kBatch2) & 1;
+        stage_ready(ka, nb, buf);
+        if (ka + kBatch2 < nAw) stage_issue(ka + kBatch2, min(kBatch2, nAw - ka - kBatch2), buf ^ 1);
 #pragma unroll 2
-        for (int k = 0; k < nb; ++k) decode_approx(k);
+        for (int k = 0; k < nb; ++k) decode_approx(k, buf);
       }
-      // int4: 8 rows per word, nibble of row k at bits 4k, stored as u = q + 8. Rotations by
-      // 17, 25, 1, 9 bring rows (0,1), (2,3), (4,5), (6,7) to mantissa bits 15 and 19:
-      // values 256 + u and 16 + u. A staged half-record is the warp's 256 bytes of nibbles
-      // followed by the record's 16 bytes of scales (17 chunks of 16 B).
-      for (int kf = 0; kf < nFw; kf += kBatch4) {
-        const int nb = min(kBatch4, nFw - kf);
-        __syncwarp();
-        uint4 v[9];
-#pragma unroll
-        for (int t = 0; t < 9; ++t) {
-          const int q = t * 32 + lane, k = q / 17, piece = q - 17 * k;
-          const int col = k < nb ? max(colF(cg + CG * (kf + k)), 0) : 0;
-          const uint8_t* src = p.full + col * p.full_col_stride;
-          v[t] = (q < 17 * kBatch4 && k < nb)
-                     ? ld_stream128(piece < 16 ? src + nib0 + 16 * piece : src + scl0)
-                     : make_uint4(0u, 0u, 0u, 0u);
+      // int4: 8 rows per word, nibble of row k at bits 4k, stored as u = q + 8. Shifts bring rows
+      // (0,1), (2,3), (4,5), (6,7) to mantissa bits 15 and 19: values 256 + u and 16 + u. A staged
+      // half-record is the warp's 256 bytes of nibbles followed by the record's 16 bytes of
+      // scales (17 chunks of 16 B); batches of kBatch4 are double-buffered by cp.async in the
+      // staging area, the next one in flight while the current one is decoded.
+      auto stage4_issue = [&](int k0, int nb, int buf) {
+        __syncwarp();  // every lane is done with what this buffer held
+        const uint32_t dst = stage_s + kStage4Bytes * buf;
+        for (int q = lane; q < nb * 17; q += 32) {
+          const int k = q / 17, piece = q - 17 * k;
+          const int col = max(colF(cg + CG * (k0 + k)), 0);
+          const uint8_t* src = p.full + col * p.full_col_stride + (piece < 16 ? nib0 + 16 * piece : scl0);
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + 16 * q), "l"(src)
+                       : "memory");
         }
-        float xk = 0.f;
-        if (lane < nb) {
-          const int i = cg + CG * (kf + lane), col = colF(i);
-          xk = col >= 0 ? xF(i, col) : 0.f;
-        }
-#pragma unroll
-        for (int t = 0; t < 9; ++t)
-          if (t * 32 + lane < 17 * kBatch4) reinterpret_cast<uint4*>(stage)[t * 32 + lane] = v[t];
+        asm volatile("cp.async.commit_group;" ::: "memory");
+      };
+      auto stage4_ready = [&](int k0, int nb, int buf) {
+        asm volatile("cp.async.wait_all;" ::: "memory");
         __syncwarp();
         if (lane < nb) {
+          const int i = cg + CG * (k0 + lane), col = colF(i);
+          const float xk = col >= 0 ? xF(i, col) : 0.f;  // an invalid column contributes zero
           // this half's four group scales: bf16 scales [4*half4, 4*half4 + 4) of the record
-          const uint2 sw = lds64(stage_s + 272 * lane + 256 + 8 * half4);
+          const uint2 sw = lds64(stage_s + kStage4Bytes * buf + 272 * lane + 256 + 8 * half4);
           const uint32_t w[4] = {sw.x << 16, sw.x & 0xFFFF0000u, sw.y << 16, sw.y & 0xFFFF0000u};
           float c[4];
 #pragma unroll
@@ -594,22 +560,33 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
             c[g] = xk * __uint_as_float(w[g]);
             s4[g] += c[g];
           }
-          asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(coef_s + 16 * lane),
-                       "f"(c[0]), "f"(c[1]), "f"(c[2]), "f"(c[3]));
+          asm volatile("st.shared.v4.f32 [%0], {%1, %1, %2, %2};" ::"r"(coef_s + 32 * lane),
+                       "f"(c[0]), "f"(c[1]));
+          asm volatile("st.shared.v4.f32 [%0], {%1, %1, %2, %2};" ::"r"(coef_s + 32 * lane + 16),
+                       "f"(c[2]), "f"(c[3]));
         }
         __syncwarp();
+      };
+      if (nFw > 0) stage4_issue(0, min(kBatch4, nFw), 0);
+      for (int kf = 0; kf < nFw; kf += kBatch4) {
+        const int nb = min(kBatch4, nFw - kf), buf = (kf / kBatch4) & 1;
+        stage4_ready(kf, nb, buf);
+        if (kf + kBatch4 < nFw) stage4_issue(kf + kBatch4, min(kBatch4, nFw - kf - kBatch4), buf ^ 1);
 #pragma unroll 2
         for (int k = 0; k < nb; ++k) {
-          const uint32_t rec = stage_s + 272 * k;
+          const uint32_t rec = stage_s + kStage4Bytes * buf + 272 * k;
           const uint32_t n0 = lds32(rec + 4 * lane), n1 = lds32(rec + 128 + 4 * lane);
-          const float c0 = __uint_as_float(lds32(coef_s + 16 * k + 4 * (lane / 16)));
-          const float c1 = __uint_as_float(lds32(coef_s + 16 * k + 4 * (2 + lane / 16)));
+          const uint2 p0 = lds64(coef_s + 32 * k + 8 * (lane / 16));
+          const uint2 p1 = lds64(coef_s + 32 * k + 8 * (2 + lane / 16));
 #pragma unroll
           for (int b = 0; b < 2; ++b) {
             const uint32_t w = b ? n1 : n0;
-            const f2 c2 = b ? f2{c1, c1} : f2{c0, c0};
-            const uint32_t rA = __funnelshift_r(w, w, 17), rB = __funnelshift_r(w, w, 25);
-            const uint32_t rC = __funnelshift_r(w, w, 1), rD = __funnelshift_r(w, w, 9);
+            const uint2 pc = b ? p1 : p0;
+            const f2 c2{__uint_as_float(pc.x), __uint_as_float(pc.y)};
+            // shifts left by 15 and 7 as multiplies, right by 1 and 9 as the high words of
+            // multiplies
+            const uint32_t rA = w * 32768u, rB = w * 128u;
+            const uint32_t rC = __umulhi(w, 0x80000000u), rD = __umulhi(w, 0x00800000u);
             acc[4 * b + 0] = ffma2(f2{code_f(rA, 0xFu << 15, 0x43800000u), code_f(rA, 0xFu << 19, 0x41800000u)}, c2, acc[4 * b + 0]);
             acc[4 * b + 1] = ffma2(f2{code_f(rB, 0xFu << 15, 0x43800000u), code_f(rB, 0xFu << 19, 0x41800000u)}, c2, acc[4 * b + 1]);
             acc[4 * b + 2] = ffma2(f2{code_f(rC, 0xFu << 15, 0x43800000u), code_f(rC, 0xFu << 19, 0x41800000u)}, c2, acc[4 * b + 2]);
