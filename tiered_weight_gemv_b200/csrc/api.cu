@@ -274,6 +274,42 @@ spax_status spax_masked_gemv_wina(const spax_packed* W, const float* x, const fl
                             status, ws, ws_bytes, stream);
 }
 
+spax_status spax_output_change(const float* y, const float* y_ref, int n, double* acc,
+                               void* stream) {
+  if (!y || !y_ref || !acc) return SPAX_ERR_ARG;
+  if (n < 1) return SPAX_ERR_SHAPE;
+  return launch_status(launch_output_change(y, y_ref, n, acc, static_cast<cudaStream_t>(stream)));
+}
+
+spax_status spax_probe_sensitivity(const spax_packed* W, const float* X, int n_tok, int s_probe_bp,
+                                   float* y2, double* acc, int32_t* status, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  if (!W || !X || !y2 || !acc) return SPAX_ERR_ARG;
+  if (n_tok < 1) return SPAX_ERR_SHAPE;
+  if (s_probe_bp < 0 || s_probe_bp > 10000) return SPAX_ERR_ARG;
+  const int d = W->d_in, d_out = W->d_out;
+  const int skip = (int)(((long long)s_probe_bp * d + 5000) / 10000);
+  spax_mask_params all = {}, probe = {};
+  all.mode = probe.mode = SPAX_MASK_TOPK;
+  all.k_full = d;                 // the reference: every column in full
+  probe.k_full = d - skip;        // the probe: the skip smallest |x| left out, the rest in full
+  float* y_ref = y2;
+  float* y = y2 + d_out;
+  if (reinterpret_cast<uintptr_t>(y) & 15u) return SPAX_ERR_ARG;
+  for (int t = 0; t < n_tok; ++t) {
+    const float* x = X + (size_t)t * d;
+    spax_status st = masked_gemv_common(W, x, false, nullptr, nullptr, &all, y_ref, nullptr,
+                                        nullptr, nullptr, nullptr, status, ws, ws_bytes, stream);
+    if (st != SPAX_OK) return st;
+    st = masked_gemv_common(W, x, false, nullptr, nullptr, &probe, y, nullptr, nullptr, nullptr,
+                            nullptr, status, ws, ws_bytes, stream);
+    if (st != SPAX_OK) return st;
+    st = launch_status(launch_output_change(y, y_ref, d_out, acc, static_cast<cudaStream_t>(stream)));
+    if (st != SPAX_OK) return st;
+  }
+  return SPAX_OK;
+}
+
 spax_status spax_column_norms(const void* W, int d_out, int d_in, float* norms, void* stream) {
   if (!W || !norms) return SPAX_ERR_ARG;
   if (d_out < 1 || d_in < 1) return SPAX_ERR_SHAPE;

@@ -141,4 +141,43 @@ cudaError_t launch_calibrate(const float* X, long long M, long long idx_skip, lo
   return cudaSuccess;
 }
 
+// ---- output change of a sparsified projection (the sensitivity probe) -------------------------
+// acc[0] += Σ_i (y_i - y_ref_i)^2, acc[1] += Σ_i y_ref_i^2 in fp64, by one CTA in a fixed order
+// (strided per-thread sums, then a fixed tree), so the result does not depend on timing.
+constexpr int kChangeThreads = 512;
+
+__global__ void __launch_bounds__(kChangeThreads)
+    output_change_kernel(const float* __restrict__ y, const float* __restrict__ y_ref, int n,
+                         double* acc) {
+  __shared__ double s0[kChangeThreads / 32], s1[kChangeThreads / 32];
+  pdl_wait();
+  pdl_launch_dependents();
+  double a = 0.0, b = 0.0;
+  for (int i = threadIdx.x; i < n; i += kChangeThreads) {
+    const double r = (double)y_ref[i], e = (double)y[i] - r;
+    a = fma(e, e, a);
+    b = fma(r, r, b);
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    a += __shfl_xor_sync(0xffffffffu, a, o);
+    b += __shfl_xor_sync(0xffffffffu, b, o);
+  }
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  if (lane == 0) s0[wid] = a, s1[wid] = b;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double ta = 0.0, tb = 0.0;
+    for (int w = 0; w < kChangeThreads / 32; ++w) ta += s0[w], tb += s1[w];
+    acc[0] += ta;
+    acc[1] += tb;
+  }
+}
+
+cudaError_t launch_output_change(const float* y, const float* y_ref, int n, double* acc,
+                                 cudaStream_t stream) {
+  return launch_pdl(output_change_kernel, dim3(1), dim3(kChangeThreads), 0, stream, y, y_ref, n,
+                    acc);
+}
+
 }  // namespace spax

@@ -93,9 +93,21 @@ struct GemvParams {
 };
 
 // Code -> float: (word & (mask << p)) | bits(C) is the float C + code, exactly, when C = 2^(23-p)
-// (the code lands in the mantissa bits whose weight is 1).
-__device__ __forceinline__ float code_f(uint32_t rot, uint32_t mask_at_p, uint32_t c_bits) {
-  return __uint_as_float((rot & mask_at_p) | c_bits);
+// (the code lands in the mantissa bits whose weight is 1). Written as one LOP3 with the mask
+// immediate and bits(C) in a register: with both operands immediate the compiler splits it into
+// two integer-pipe instructions (measured: 32 instead of 16 per 512-row 2-bit column segment).
+template <uint32_t MASK>
+__device__ __forceinline__ float code_f(uint32_t rot, uint32_t c_bits) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(rot), "n"(MASK), "r"(c_bits));  // (a&b)|c
+  return __uint_as_float(d);
+}
+// bits(C) for C = 256, 64, 16, 4, held in registers (an opaque move keeps the compiler from
+// folding them back into immediates)
+__device__ __forceinline__ uint32_t reg_const(uint32_t v) {
+  uint32_t r;
+  asm volatile("mov.b32 %0, %1;" : "=r"(r) : "r"(v));
+  return r;
 }
 
 // Index of row r inside a combine slot (36 floats per 32 rows: padding spreads the banks).
@@ -170,6 +182,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int tile = blockIdx.x, split = blockIdx.y, S = p.S;
+  // the decode constants (none in the dense GEMV)
+  const uint32_t kC256 = DENSE ? 0u : reg_const(0x43800000u), kC64 = DENSE ? 0u : reg_const(0x42800000u);
+  const uint32_t kC16 = DENSE ? 0u : reg_const(0x41800000u), kC4 = DENSE ? 0u : reg_const(0x40800000u);
   const int r0 = tile * R;
   const int rows_here = min(R, p.d_out - r0);
   const int rg = warp / CG, cg = warp % CG;
@@ -348,10 +363,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
       const uint2 pc = b ? p1 : p0;
       const f2 c2{__uint_as_float(pc.x), __uint_as_float(pc.y)};
       const uint32_t ra = w * 32768u, rc = w * 128u;
-      acc[4 * b + 0] = ffma2(f2{code_f(ra, 3u << 15, 0x43800000u), code_f(ra, 3u << 17, 0x42800000u)}, c2, acc[4 * b + 0]);
-      acc[4 * b + 1] = ffma2(f2{code_f(ra, 3u << 19, 0x41800000u), code_f(ra, 3u << 21, 0x40800000u)}, c2, acc[4 * b + 1]);
-      acc[4 * b + 2] = ffma2(f2{code_f(rc, 3u << 15, 0x43800000u), code_f(rc, 3u << 17, 0x42800000u)}, c2, acc[4 * b + 2]);
-      acc[4 * b + 3] = ffma2(f2{code_f(rc, 3u << 19, 0x41800000u), code_f(rc, 3u << 21, 0x40800000u)}, c2, acc[4 * b + 3]);
+      acc[4 * b + 0] = ffma2(f2{code_f<(3u << 15)>(ra, kC256), code_f<(3u << 17)>(ra, kC64)}, c2, acc[4 * b + 0]);
+      acc[4 * b + 1] = ffma2(f2{code_f<(3u << 19)>(ra, kC16), code_f<(3u << 21)>(ra, kC4)}, c2, acc[4 * b + 1]);
+      acc[4 * b + 2] = ffma2(f2{code_f<(3u << 15)>(rc, kC256), code_f<(3u << 17)>(rc, kC64)}, c2, acc[4 * b + 2]);
+      acc[4 * b + 3] = ffma2(f2{code_f<(3u << 19)>(rc, kC16), code_f<(3u << 21)>(rc, kC4)}, c2, acc[4 * b + 3]);
     }
   };
 
@@ -587,10 +602,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
             // multiplies
             const uint32_t rA = w * 32768u, rB = w * 128u;
             const uint32_t rC = __umulhi(w, 0x80000000u), rD = __umulhi(w, 0x00800000u);
-            acc[4 * b + 0] = ffma2(f2{code_f(rA, 0xFu << 15, 0x43800000u), code_f(rA, 0xFu << 19, 0x41800000u)}, c2, acc[4 * b + 0]);
-            acc[4 * b + 1] = ffma2(f2{code_f(rB, 0xFu << 15, 0x43800000u), code_f(rB, 0xFu << 19, 0x41800000u)}, c2, acc[4 * b + 1]);
-            acc[4 * b + 2] = ffma2(f2{code_f(rC, 0xFu << 15, 0x43800000u), code_f(rC, 0xFu << 19, 0x41800000u)}, c2, acc[4 * b + 2]);
-            acc[4 * b + 3] = ffma2(f2{code_f(rD, 0xFu << 15, 0x43800000u), code_f(rD, 0xFu << 19, 0x41800000u)}, c2, acc[4 * b + 3]);
+            acc[4 * b + 0] = ffma2(f2{code_f<(0xFu << 15)>(rA, kC256), code_f<(0xFu << 19)>(rA, kC16)}, c2, acc[4 * b + 0]);
+            acc[4 * b + 1] = ffma2(f2{code_f<(0xFu << 15)>(rB, kC256), code_f<(0xFu << 19)>(rB, kC16)}, c2, acc[4 * b + 1]);
+            acc[4 * b + 2] = ffma2(f2{code_f<(0xFu << 15)>(rC, kC256), code_f<(0xFu << 19)>(rC, kC16)}, c2, acc[4 * b + 2]);
+            acc[4 * b + 3] = ffma2(f2{code_f<(0xFu << 15)>(rD, kC256), code_f<(0xFu << 19)>(rD, kC16)}, c2, acc[4 * b + 3]);
           }
         }
       }

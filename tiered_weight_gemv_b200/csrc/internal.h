@@ -62,6 +62,8 @@ cudaError_t launch_column_norms(const void* W, int d_out, int d_in, float* norms
 uint8_t* fixed_scratch_current_device_ptr(size_t* bytes);
 
 size_t calibrate_ws_bytes();
+cudaError_t launch_output_change(const float* y, const float* y_ref, int n, double* acc,
+                                 cudaStream_t stream);
 cudaError_t launch_calibrate(const float* X, long long M, long long idx_skip, long long idx_full,
                              float* t_out, int32_t* status, void* ws, cudaStream_t stream);
 

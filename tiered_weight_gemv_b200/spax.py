@@ -70,6 +70,9 @@ _SIGS = {
                                        _I),
     "spax_fixed_scratch_bytes": ([], _Z),
     "spax_fixed_scratch_reset": ([_P], _I),
+    "spax_output_change": ([_P, _P, _I, _P, _P], _I),
+    "spax_probe_sensitivity": ([ctypes.POINTER(spax_packed), _P, _I, _I, _P, _P, _P, _P, _Z, _P],
+                               _I),
     "spax_test_tiered_gemv_timeout": ([ctypes.POINTER(spax_packed), _P, _P, _P, _P, _P, _P, _P, _Z,
                                       ctypes.c_uint64, _P], _I),
     "spax_workspace_bytes": ([_I, _I, _I], _Z),
@@ -376,6 +379,32 @@ def spax_test_tiered_gemv_timeout(W: PackedMatrix, x: torch.Tensor, full_idx: to
         _dev(y, torch.float32, "y"), _dev(status, torch.int32, "status"),
         None if ws is None else _dev(ws, None, "ws"),
         0 if ws is None else ws.numel() * ws.element_size(), int(wait_limit_ns),
+        _stream(stream)))
+
+
+def spax_output_change(y: torch.Tensor, y_ref: torch.Tensor, acc: torch.Tensor,
+                       stream=None) -> None:
+    """acc[0] += sum (y - y_ref)^2, acc[1] += sum y_ref^2 (fp64 device accumulators)."""
+    if y.numel() != y_ref.numel() or acc.numel() < 2:
+        raise ValueError("sizes do not match")
+    _check("spax_output_change", _lib.spax_output_change(
+        _dev(y, torch.float32, "y"), _dev(y_ref, torch.float32, "y_ref"), y.numel(),
+        _dev(acc, torch.float64, "acc"), _stream(stream)))
+
+
+def spax_probe_sensitivity(W: PackedMatrix, X: torch.Tensor, s_probe_bp: int, y2: torch.Tensor,
+                           acc: torch.Tensor, status: torch.Tensor, ws: torch.Tensor, stream=None,
+                           desc=None) -> None:
+    """Output change of one matrix at probe sparsity s_probe_bp / 1e4 over the calibration
+    tokens X [n_tok, d_in], accumulated into acc (two fp64 on the device)."""
+    n_tok, d_in = X.shape
+    if d_in != W.d_in or y2.numel() < 2 * W.d_out or acc.numel() < 2:
+        raise ValueError("sizes do not match W")
+    d = W.desc() if desc is None else desc
+    _check("spax_probe_sensitivity", _lib.spax_probe_sensitivity(
+        ctypes.byref(d), _dev(X, torch.float32, "X"), n_tok, s_probe_bp,
+        _dev(y2, torch.float32, "y2"), _dev(acc, torch.float64, "acc"),
+        _dev(status, torch.int32, "status"), _dev(ws, None, "ws"), ws.numel() * ws.element_size(),
         _stream(stream)))
 
 
