@@ -494,6 +494,15 @@ def run_gpu(args, rank, world, local):
 LLAMA3_SITES = [("qkv", 6144, 4096, 201), ("o", 4096, 4096, 202), ("gate_up", 28672, 4096, 203),
                 ("down", 4096, 14336, 204)]
 LLAMA3_POINTS = [(f, a) for f in (0.1, 0.2, 0.3) for a in (0.2, 0.3)]
+LLAMA3_LAYERS, LLAMA3_TOKENS = 32, 256
+GUIDED_TARGETS = (0.3, 0.5, 0.7)
+GUIDED_DELTA_BP = 100
+N_GUIDED_CAL = 512  # calibration tokens per (layer, site) for the guided thresholds
+N_SENS_CAL = 16     # calibration tokens per (layer, site) for the measured sensitivity
+S_PROBE_BP = 5000   # probe sparsity of the sensitivity pass
+L70_SITES = [("gate_up", 2 * 28672, 8192, 401), ("down", 8192, 28672, 402)]
+L70_TOKENS = 128
+L70_SPLITS = [(0.5, 0.25, 0.25), (0.7, 0.15, 0.15)]  # skip / approx / full
 L2_BYTES = 126 * 2 ** 20
 
 
@@ -502,165 +511,376 @@ def _replicas_for(bytes_per_replica: float) -> int:
     return max(4, math.ceil(3 * L2_BYTES / bytes_per_replica))
 
 
-def run_extras(args, dev):
-    """Measurements beside the headline, on one GPU (each a CUDA graph of n tokens, timed like the
-    headline): dequantisation against loading, the Llama-3-8B (full, approx) sweep with its
-    c0 + bytes/BW fit, and the dense kernels (this library's and torch.mv / cuBLAS) on the same
-    layer."""
+def _k(frac: float, d: int) -> int:
+    return int(math.floor(frac * d + 0.5))
+
+
+def _timed_graph(fn, stream, steps, warmup):
+    """Run fn once eagerly, capture it as one CUDA graph and time its replays (ms per replay)."""
+    with torch.cuda.stream(stream):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    ms = time_graph(g, steps, warmup, stream)
+    del g
+    return ms
+
+
+def run_dequant(args, dev):
+    """Dequantisation against loading on 4096x4096 and 22016x4096: all-bf16, all-2-bit, mixed
+    25/25 and all-2-bit on one L2-resident weight copy, each through the masked GEMV and through
+    the list-driven GEMV on lists built beforehand (no selection in the timed launches). The
+    list-driven all-2-bit L2-resident case is the decode's own cost, without HBM or selection."""
     from tiered_weight_gemv_b200 import spax, synth
 
     n_tok = 16
     steps, warmup = max(5, min(args.steps, 20)), args.warmup
     stream = torch.cuda.Stream(device=dev)
     out = {}
-
-    def packed_replicas(W, d_out, d_in, n_rep):
-        pm = spax.alloc_packed(d_out, d_in, spax.FULL_BF16, device=dev)
-        spax.spax_pack_weights(W, spax.FULL_BF16, pm)
-        return [pm] + [spax.PackedMatrix(d_out, d_in, spax.FULL_BF16, pm.full.clone(),
-                                         pm.approx.clone()) for _ in range(n_rep - 1)]
-
-    def timed(fn):
-        with torch.cuda.stream(stream):
-            fn()
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            fn()
-        ms = time_graph(g, steps, warmup, stream)
-        del g
-        return ms
-
-    # ---- dequantisation against loading: all bf16, all 2-bit, mixed, 2-bit from L2 ----
-    dq = {}
     for label, d_out, d_in, tid in [("proj_4096x4096", 4096, 4096, 301),
                                     ("gate_up_22016x4096", 22016, 4096, 302)]:
         W = synth.weight(d_out, d_in, 6, tid, device=dev)
-        reps = packed_replicas(W, d_out, d_in, _replicas_for(2.3 * d_out * d_in))
+        pm = spax.alloc_packed(d_out, d_in, spax.FULL_BF16, device=dev)
+        spax.spax_pack_weights(W, spax.FULL_BF16, pm)
+        reps = [pm] + [spax.PackedMatrix(d_out, d_in, spax.FULL_BF16, pm.full.clone(), pm.approx.clone())
+                       for _ in range(_replicas_for(2.3 * d_out * d_in) - 1)]
         del W
         X = synth.laplace((n_tok, d_in), 6, tid + 10, device=dev)
         y = torch.empty(n_tok, d_out, device=dev)
         st = torch.zeros(1, dtype=torch.int32, device=dev)
         ws = spax.alloc_workspace(spax.OP_TIERED_GEMV, d_out, d_in, device=dev)
-        descs = [pm.desc() for pm in reps]
-        q = int(math.floor(0.25 * d_in + 0.5))
-        cases = [("all_full", d_in, 0, True), ("all_approx", 0, d_in, True),
-                 ("mixed_25_25", q, q, True), ("all_approx_l2_resident", 0, d_in, False)]
+        descs = [r.desc() for r in reps]
+        tier = torch.empty(n_tok, d_in, dtype=torch.uint8, device=dev)
+        fi = torch.empty(n_tok, d_in, dtype=torch.int32, device=dev)
+        ai = torch.empty(n_tok, d_in, dtype=torch.int32, device=dev)
+        cnt = torch.empty(n_tok, 4, dtype=torch.int32, device=dev)
+        q = _k(0.25, d_in)
         rows = {}
-        for case, kf, ka, rotate in cases:
+        for case, kf, ka, rotate in [("all_full", d_in, 0, True), ("all_approx", 0, d_in, True),
+                                     ("mixed_25_25", q, q, True),
+                                     ("all_approx_l2_resident", 0, d_in, False)]:
             prm = spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka)
+            for t in range(n_tok):  # the lists of the list-driven arm, built outside the timing
+                spax.spax_build_mask(X[t], prm, tier[t], fi[t], ai[t], cnt[t], st)
 
-            def fn(prm=prm, rotate=rotate):
+            def masked(prm=prm, rotate=rotate):
                 for t in range(n_tok):
                     r = t % len(reps) if rotate else 0
                     spax.spax_masked_gemv(reps[r], X[t], prm, y[t], st, ws, desc=descs[r])
 
-            ms = timed(fn)
+            def listed(rotate=rotate):
+                for t in range(n_tok):
+                    r = t % len(reps) if rotate else 0
+                    spax.spax_tiered_gemv(reps[r], X[t], fi[t], ai[t], cnt[t], y[t], st, ws,
+                                          desc=descs[r])
+
+            ms = _timed_graph(masked, stream, steps, warmup)
+            ms_l = _timed_graph(listed, stream, steps, warmup)
             by = fused_bytes(d_out, d_in, kf, ka)
-            rows[case] = {"us": round(ms * 1000 / n_tok, 3), "bytes": by,
-                          "GBps": round(by * n_tok / (ms * 1e-3) / 1e9, 1)}
+            by_l = algorithmic_bytes(d_out, d_in, kf, ka)
+            rows[case] = {"masked_us": round(ms * 1000 / n_tok, 3), "masked_bytes": by,
+                          "masked_GBps": round(by * n_tok / (ms * 1e-3) / 1e9, 1),
+                          "list_driven_us": round(ms_l * 1000 / n_tok, 3), "list_driven_bytes": by_l,
+                          "list_driven_GBps": round(by_l * n_tok / (ms_l * 1e-3) / 1e9, 1),
+                          "selection_us": round((ms - ms_l) * 1000 / n_tok, 3)}
         if int(st.item()) != 0:
             raise RuntimeError(f"device status {int(st.item())} in the dequant runs ({label})")
         rows["replicas"] = len(reps)
-        dq[label] = rows
-        del reps, descs, ws, X, y
+        out[label] = rows
+        del reps, descs, ws, X, y, tier, fi, ai, cnt
         torch.cuda.empty_cache()
-    out["dequant_vs_load"] = dq
+    out["note"] = ("list_driven_* time spax_tiered_gemv on lists built beforehand (no selection in "
+                   "the timed launches); selection_us = masked - list-driven; the all-2-bit "
+                   "L2-resident list-driven case is the 2-bit decode's own cost")
+    return out
 
-    # ---- Llama-3-8B layer: the six (full, approx) points, dense, torch.mv ----
-    per_rep = sum(2.3 * d_out * d_in for _, d_out, d_in, _ in LLAMA3_SITES)
-    n_rep = _replicas_for(per_rep)
-    layer = {}
-    for name, d_out, d_in, tid in LLAMA3_SITES:
-        W = synth.weight(d_out, d_in, 7, tid, device=dev)
-        reps = packed_replicas(W, d_out, d_in, n_rep)
-        del W
-        layer[name] = dict(reps=reps, descs=[pm.desc() for pm in reps],
-                           X=synth.laplace((n_tok, d_in), 7, tid + 10, device=dev),
-                           y=torch.empty(n_tok, d_out, device=dev),
-                           st=torch.zeros(1, dtype=torch.int32, device=dev),
-                           ws=spax.alloc_workspace(spax.OP_TIERED_GEMV, d_out, d_in, device=dev),
-                           dws=spax.alloc_workspace(spax.OP_DENSE_GEMV, d_out, d_in, device=dev))
-        layer[name]["Xh"] = layer[name]["X"].to(torch.bfloat16)
-        # calibration tokens of the site's own distribution, never timed (the boundary guesses)
-        layer[name]["cal"] = synth.laplace((N_CAL, d_in), 8, tid + 10, device=dev)
-        layer[name]["cal_ws"] = torch.empty(spax.spax_workspace_bytes(spax.OP_CALIBRATE, 0, d_in),
-                                            dtype=torch.uint8, device=dev)
+
+def run_llama3_stack(args, dev):
+    """The Llama-3-8B-shaped projection stack at its stated size: 32 layers with their own
+    seeded weights, 256 tokens of Laplace activations per site and layer, every launch on weights
+    no other launch of the step shares (6.5 GB of packed pools: L2-cold).
+      * The (full, approx) sweep with TopK masks, with and without calibrated boundary-key
+        guesses, and its fit time = c0 + bytes/BW (the ByteCross abstract's method).
+      * The dense GEMV and torch.mv (cuBLAS) over the same stack.
+      * The measured block sensitivity (TopK-Guided §2.2) at probe sparsity 0.5 on calibration
+        tokens, and the TopK-Guided masks at targets 0.3 / 0.5 / 0.7 (±0.01): per-layer
+        thresholds calibrated on 512 tokens, per-block budgets (λ = 0.5, clamp [0.05, 0.95])
+        from the synthetic profile and from the measured sensitivity; bytes counted from the
+        realised lists of every launch."""
+    from tiered_weight_gemv_b200 import spax, synth
+
+    L, T = LLAMA3_LAYERS, LLAMA3_TOKENS
+    steps, warmup = 3, args.warmup
+    stream = torch.cuda.Stream(device=dev)
+    names = [s[0] for s in LLAMA3_SITES]
+    pm, X = {}, {}
+    for l in range(L):
+        for name, d_out, d_in, tid in LLAMA3_SITES:
+            W = synth.weight(d_out, d_in, 7, 1000 * l + tid, device=dev)
+            p = spax.alloc_packed(d_out, d_in, spax.FULL_BF16, device=dev)
+            spax.spax_pack_weights(W, spax.FULL_BF16, p)
+            pm[l, name] = p
+            X[l, name] = synth.laplace((T, d_in), 7, 100000 + 1000 * l + tid, device=dev)
+            del W
     torch.cuda.synchronize()
-    t_cal = torch.empty(2, device=dev)
-    st_cal = torch.zeros(1, dtype=torch.int32, device=dev)
+    desc = {k: v.desc() for k, v in pm.items()}
+    shape = {name: (d_out, d_in) for name, d_out, d_in, _ in LLAMA3_SITES}
+    ws = {n: spax.alloc_workspace(spax.OP_TIERED_GEMV, *shape[n], device=dev) for n in names}
+    dws = {n: spax.alloc_workspace(spax.OP_DENSE_GEMV, *shape[n], device=dev) for n in names}
+    y = {n: torch.empty(T, shape[n][0], device=dev) for n in names}
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    cal_ws = {n: torch.empty(spax.spax_workspace_bytes(spax.OP_CALIBRATE, 0, shape[n][1]),
+                             dtype=torch.uint8, device=dev) for n in names}
+    t2 = torch.empty(2, device=dev)
+
+    def calibrate(cal, d_in, s_skip, s_below_full, name):
+        spax.spax_calibrate_thresholds(cal, round(s_skip * 10000), round(s_below_full * 10000), t2,
+                                       st, cal_ws[name])
+        return tuple(float(v) for v in t2.cpu())
+
+    def run_masked(prm):
+        for t in range(T):
+            for l in range(L):
+                for n in names:
+                    spax.spax_masked_gemv(pm[l, n], X[l, n][t], prm[l, n], y[n][t], st, ws[n],
+                                          desc=desc[l, n])
+
+    out = {"layers": L, "tokens": T, "sites": {n: list(shape[n]) for n in names},
+           "packed_GB": round(sum(v.full.numel() + v.approx.numel() for v in pm.values()) / 1e9, 2)}
+    # ---- config 3: the (full, approx) sweep ----
+    guess_cal = {(l, n): synth.laplace((N_CAL, shape[n][1]), 8, 200000 + 1000 * l + i, device=dev)
+                 for l in range(L) for i, n in enumerate(names)}
     points = []
     for f, a in LLAMA3_POINTS:
         prms, prms0 = {}, {}
-        for name, _, d_in, _ in LLAMA3_SITES:
-            kf, ka = int(math.floor(f * d_in + 0.5)), int(math.floor(a * d_in + 0.5))
-            L = layer[name]
-            spax.spax_calibrate_thresholds(L["cal"], round((d_in - kf - ka) * 10000 / d_in),
-                                           round((d_in - kf) * 10000 / d_in), t_cal, st_cal,
-                                           L["cal_ws"])
-            t_skip, t_full = (float(v) for v in t_cal.cpu())
-            prms[name] = spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka, t_skip=t_skip,
-                                          t_full=t_full)
-            prms0[name] = spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka)
-        if int(st_cal.item()) != 0:
-            raise RuntimeError(f"calibration status {int(st_cal.item())} in the sweep")
+        for l in range(L):
+            for n in names:
+                d_in = shape[n][1]
+                kf, ka = _k(f, d_in), _k(a, d_in)
+                ts, tf = calibrate(guess_cal[l, n], d_in, (d_in - kf - ka) / d_in, (d_in - kf) / d_in, n)
+                prms[l, n] = spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka, t_skip=ts, t_full=tf)
+                prms0[l, n] = spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka)
+        ms = _timed_graph(lambda: run_masked(prms), stream, steps, warmup)
+        ms0 = _timed_graph(lambda: run_masked(prms0), stream, steps, warmup)
+        by = sum(fused_bytes(*shape[n], _k(f, shape[n][1]), _k(a, shape[n][1])) for n in names)
+        us = ms * 1000 / (T * L)
+        points.append({"full": f, "approx": a, "us_per_token_layer": round(us, 3),
+                       "unguessed_us_per_token_layer": round(ms0 * 1000 / (T * L), 3),
+                       "bytes_per_token_layer": by, "GBps": round(by / (us * 1e-6) / 1e9, 1),
+                       "frac_of_8TBps": round(by / (us * 1e-6) / 8e12, 4)})
+    del guess_cal
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} in the Llama-3 sweep")
+    out["points"] = points
+    out["fit_time_vs_bytes"] = fit_c0_bw([(p["bytes_per_token_layer"], p["us_per_token_layer"]) for p in points])
+    out["unguessed_fit_time_vs_bytes"] = fit_c0_bw([(p["bytes_per_token_layer"], p["unguessed_us_per_token_layer"]) for p in points])
+    out["guess_note"] = ("the TopK parameters carry |x| quantiles calibrated on 16 separate tokens per "
+                         "layer, site and point; unguessed_* is the same launches without them")
 
-        def fn(prms):
-            for t in range(n_tok):
-                for name, *_ in LLAMA3_SITES:
-                    L = layer[name]
-                    r = t % n_rep
-                    spax.spax_masked_gemv(L["reps"][r], L["X"][t], prms[name], L["y"][t], L["st"],
-                                          L["ws"], desc=L["descs"][r])
+    def run_dense():
+        for t in range(T):
+            for l in range(L):
+                for n in names:
+                    spax.spax_dense_gemv(pm[l, n].full, X[l, n][t], y[n][t], *shape[n], st, dws[n])
 
-        ms = timed(lambda: fn(prms))
-        ms0 = timed(lambda: fn(prms0))
-        by = sum(fused_bytes(d_out, d_in, prms[n].k_full, prms[n].k_approx)
-                 for n, d_out, d_in, _ in LLAMA3_SITES)
-        points.append({"full": f, "approx": a, "us_per_token_layer": round(ms * 1000 / n_tok, 3),
-                       "unguessed_us_per_token_layer": round(ms0 * 1000 / n_tok, 3),
-                       "bytes_per_token_layer": by,
-                       "GBps": round(by * n_tok / (ms * 1e-3) / 1e9, 1)})
-    for name, *_ in LLAMA3_SITES:
-        if int(layer[name]["st"].item()) != 0:
-            raise RuntimeError(f"device status {int(layer[name]['st'].item())} in the sweep ({name})")
+    Xh = {k: v.to(torch.bfloat16) for k, v in X.items()}
 
-    def dense_fn():
-        for t in range(n_tok):
-            for name, d_out, d_in, _ in LLAMA3_SITES:
-                L = layer[name]
-                spax.spax_dense_gemv(L["reps"][t % n_rep].full, L["X"][t], L["y"][t], d_out, d_in,
-                                     L["st"], L["dws"])
+    def run_mv():
+        for t in range(T):
+            for l in range(L):
+                for n in names:
+                    d_out, d_in = shape[n]
+                    torch.mv(pm[l, n].full.view(torch.bfloat16).view(d_in, d_out).t(), Xh[l, n][t])
 
-    def torch_mv_fn():
-        for t in range(n_tok):
-            for name, d_out, d_in, _ in LLAMA3_SITES:
-                L = layer[name]
-                Wt = L["reps"][t % n_rep].full.view(torch.bfloat16).view(d_in, d_out)
-                torch.mv(Wt.t(), L["Xh"][t])
+    dense_bytes = sum(2 * d_out * d_in for d_out, d_in in shape.values())
+    ms_d = _timed_graph(run_dense, stream, steps, warmup)
+    ms_mv = _timed_graph(run_mv, stream, steps, warmup)
+    del Xh
+    out["dense_us_per_token_layer"] = round(ms_d * 1000 / (T * L), 3)
+    out["dense_GBps"] = round(dense_bytes * T * L / (ms_d * 1e-3) / 1e9, 1)
+    out["torch_mv_bf16_us_per_token_layer"] = round(ms_mv * 1000 / (T * L), 3)
+    out["torch_mv_note"] = "cuBLAS through torch.mv on the same bf16 pools with bf16 x (sanity figure)"
 
-    dense_bytes = sum(2 * d_out * d_in for _, d_out, d_in, _ in LLAMA3_SITES)
-    ms_dense = timed(dense_fn)
-    ms_mv = timed(torch_mv_fn)
-    out["llama3_8b_layer_sweep"] = {
-        "sites": {n: [d_out, d_in] for n, d_out, d_in, _ in LLAMA3_SITES},
-        "tokens": n_tok, "replicas": n_rep, "points": points,
-        "fit_time_vs_bytes": fit_c0_bw([(p["bytes_per_token_layer"], p["us_per_token_layer"])
-                                        for p in points]),
-        "unguessed_fit_time_vs_bytes": fit_c0_bw([(p["bytes_per_token_layer"],
-                                                   p["unguessed_us_per_token_layer"]) for p in points]),
-        "guess_note": "the TopK parameters carry |x| quantiles calibrated on 16 separate tokens per "
-                      "site and point; unguessed_* is the same launch sequence without them",
-        "dense_us_per_token_layer": round(ms_dense * 1000 / n_tok, 3),
-        "dense_GBps": round(dense_bytes * n_tok / (ms_dense * 1e-3) / 1e9, 1),
-        "torch_mv_bf16_us_per_token_layer": round(ms_mv * 1000 / n_tok, 3),
-        "torch_mv_note": "cuBLAS through torch.mv on the same bf16 pool with bf16 x (sanity figure)",
-    }
-    del layer
+    # ---- the measured block sensitivity (TopK-Guided §2.2) ----
+    y2 = {n: torch.empty(2 * shape[n][0], device=dev) for n in names}
+    acc = torch.zeros(L, len(names), 2, dtype=torch.float64, device=dev)
+    for l in range(L):
+        for i, n in enumerate(names):
+            cal = synth.laplace((N_SENS_CAL, shape[n][1]), 9, 300000 + 1000 * l + i, device=dev)
+            spax.spax_probe_sensitivity(pm[l, n], cal, S_PROBE_BP, y2[n], acc[l, i], st, ws[n],
+                                        desc=desc[l, n])
+    a = acc.cpu().numpy()
+    sens_meas = np.sqrt(a[:, :, 0].sum(1) / a[:, :, 1].sum(1))
+    sens_syn = 1.0 + 3.0 * np.exp(-np.arange(L) / 4.0)
+    out["sensitivity"] = {"probe_sparsity": S_PROBE_BP / 10000, "calibration_tokens": N_SENS_CAL,
+                          "measured": [round(float(v), 6) for v in sens_meas],
+                          "synthetic_profile": "1 + 3 exp(-b/4)"}
+
+    # ---- config 4: TopK-Guided masks on the stack ----
+    cnt = torch.zeros(T, L, len(names), 4, dtype=torch.int32, device=dev)
+
+    def run_guided(prm):
+        for t in range(T):
+            for l in range(L):
+                for i, n in enumerate(names):
+                    spax.spax_masked_gemv(pm[l, n], X[l, n][t], prm[l, n], y[n][t], st, ws[n],
+                                          counts=cnt[t, l, i], desc=desc[l, n])
+
+    guided = []
+    for src, sens in (("synthetic", sens_syn), ("measured", sens_meas)):
+        for s in GUIDED_TARGETS:
+            s_b = spax.spax_block_budgets(sens, s, 0.5, 0.05, 0.95)
+            prm = {}
+            for l in range(L):
+                s1 = float(s_b[l])
+                s2 = s1 + (1.0 - s1) / 2.0  # the kept budget split evenly between the tiers
+                for i, n in enumerate(names):
+                    d_in = shape[n][1]
+                    cal = synth.laplace((N_GUIDED_CAL, d_in), 10, 400000 + 1000 * l + i, device=dev)
+                    ts, tf = calibrate(cal, d_in, s1, s2, n)
+                    prm[l, n] = spax.mask_params(spax.MASK_GUIDED, t_skip=ts, t_full=tf,
+                                                 s_skip_bp=round(s1 * 10000),
+                                                 s_below_full_bp=round(s2 * 10000),
+                                                 delta_bp=GUIDED_DELTA_BP)
+                    del cal
+            ms = _timed_graph(lambda: run_guided(prm), stream, steps, warmup)
+            c = cnt.cpu().numpy().astype(np.int64)  # realised counts of the last replay
+            nbytes = 0
+            skip_dev = 0.0
+            for l in range(L):
+                for i, n in enumerate(names):
+                    d_out, d_in = shape[n]
+                    nf, na = c[:, l, i, 0], c[:, l, i, 1]
+                    nbytes += sum(fused_bytes(d_out, d_in, int(f_), int(a_)) for f_, a_ in zip(nf, na))
+                    real = (d_in - nf - na) / d_in
+                    skip_dev = max(skip_dev, float(np.max(np.abs(real - round(float(s_b[l]) * 10000) / 10000))))
+            us = ms * 1000 / (T * L)
+            bpt = nbytes / (T * L)
+            guided.append({"budgets_from": src, "target": s, "us_per_token_layer": round(us, 3),
+                           "realised_bytes_per_token_layer": round(bpt),
+                           "GBps": round(bpt / (us * 1e-6) / 1e9, 1),
+                           "frac_of_8TBps": round(bpt / (us * 1e-6) / 8e12, 4),
+                           "max_realised_skip_deviation": round(skip_dev, 5),
+                           "block_budget_range": [round(float(s_b.min()), 4), round(float(s_b.max()), 4)]})
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} in the guided runs")
+    out["topk_guided"] = guided
+    out["topk_guided_note"] = ("guided rule, delta 0.01; thresholds per layer and site from 512 "
+                               "calibration tokens; block budgets lambda 0.5, clamp [0.05, 0.95]; "
+                               "bytes from the counts each launch wrote; the skip deviation is the "
+                               "largest |realised - block target| over all launches (at most 0.01)")
+    del pm, X, desc, y, ws, dws
     torch.cuda.empty_cache()
+    return out
+
+
+def run_llama2_70b_mlp(args, dev):
+    """The Llama-2-70B-shaped MLP with the int4 full tier (group 128, symmetric) and the 2-bit
+    approximate tier: gate/up (concatenated, 57344x8192) and down (8192x28672), 128 tokens of
+    Laplace activations at each site, tiers 50/25/25 and 70/15/15 by |x| rank, against the same
+    kernel with every column in the int4 tier (dense in the same weight format)."""
+    from tiered_weight_gemv_b200 import spax, synth
+
+    T = L70_TOKENS
+    steps, warmup = max(3, min(args.steps, 10)), args.warmup
+    stream = torch.cuda.Stream(device=dev)
+    per_rep = sum(spax.spax_pack_bytes(d_out, d_in, spax.FULL_INT4_G128)[0] +
+                  spax.spax_pack_bytes(d_out, d_in, spax.FULL_INT4_G128)[1]
+                  for _, d_out, d_in, _ in L70_SITES)
+    n_rep = _replicas_for(per_rep)
+    reps, X, y, ws = {}, {}, {}, {}
+    for name, d_out, d_in, tid in L70_SITES:
+        W = synth.weight(d_out, d_in, 11, tid, device=dev)
+        p = spax.alloc_packed(d_out, d_in, spax.FULL_INT4_G128, device=dev)
+        spax.spax_pack_weights(W, spax.FULL_INT4_G128, p)
+        del W
+        torch.cuda.synchronize()
+        reps[name] = [p] + [spax.PackedMatrix(d_out, d_in, spax.FULL_INT4_G128, p.full.clone(),
+                                              p.approx.clone()) for _ in range(n_rep - 1)]
+        X[name] = synth.laplace((T, d_in), 11, tid + 10, device=dev)
+        y[name] = torch.empty(T, d_out, device=dev)
+        ws[name] = spax.alloc_workspace(spax.OP_TIERED_GEMV, d_out, d_in, device=dev)
+    desc = {n: [r.desc() for r in reps[n]] for n in reps}
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def run(split):
+        for t in range(T):
+            for name, d_out, d_in, _ in L70_SITES:
+                _, a, f = split
+                prm = spax.mask_params(spax.MASK_TOPK, k_full=_k(f, d_in), k_approx=_k(a, d_in))
+                spax.spax_masked_gemv(reps[name][t % n_rep], X[name][t], prm, y[name][t], st,
+                                      ws[name], desc=desc[name][t % n_rep])
+
+    def bytes_of(split):
+        _, a, f = split
+        return sum(spax.spax_weight_bytes(d_out, spax.FULL_INT4_G128, _k(f, d_in), _k(a, d_in)) +
+                   5 * d_in + 4 * (_k(f, d_in) + _k(a, d_in)) + 4 * d_out + 16
+                   for _, d_out, d_in, _ in L70_SITES)
+
+    out = {"sites": {n: [d_out, d_in] for n, d_out, d_in, _ in L70_SITES}, "tokens": T,
+           "replicas": n_rep, "full_tier": "int4 g128 symmetric", "splits": []}
+    dense = (0.0, 0.0, 1.0)
+    ms_dense = _timed_graph(lambda: run(dense), stream, steps, warmup)
+    for split in L70_SPLITS:
+        ms = _timed_graph(lambda: run(split), stream, steps, warmup)
+        us = ms * 1000 / T
+        by = bytes_of(split)
+        out["splits"].append({"skip": split[0], "approx": split[1], "full": split[2],
+                              "us_per_token_mlp": round(us, 3), "bytes_per_token_mlp": by,
+                              "GBps": round(by / (us * 1e-6) / 1e9, 1),
+                              "frac_of_8TBps": round(by / (us * 1e-6) / 8e12, 4),
+                              "speedup_vs_dense_int4": round(ms_dense / ms, 3)})
+    by_d = bytes_of(dense)
+    out["dense_int4_us_per_token_mlp"] = round(ms_dense * 1000 / T, 3)
+    out["dense_int4_GBps"] = round(by_d / (ms_dense * 1e-3 / T) / 1e9, 1)
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} in the 70B MLP runs")
+    del reps, desc, X, y, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_extras(args, dev):
+    """Measurements beside the headline, on one GPU, each a CUDA graph timed like the headline."""
+    out = {"dequant_vs_load": run_dequant(args, dev)}
+    out["llama3_8b_stack"] = run_llama3_stack(args, dev)
+    out["llama2_70b_mlp_int4"] = run_llama2_70b_mlp(args, dev)
     out["host_link_offload"] = run_host_link(args, dev)
     torch.cuda.empty_cache()
     return out
+
+
+def run_decode_case(args, dev):
+    """Profiling aid (no timing, no JSON line): the list-driven GEMV on 22016x4096 with every
+    column in the 2-bit tier, lists built beforehand, one L2-resident weight copy, 4 launches
+    after one mask launch. Under ncu it isolates the 2-bit decode from HBM and from the
+    selection."""
+    from tiered_weight_gemv_b200 import spax, synth
+
+    d_out, d_in = 22016, 4096
+    W = synth.weight(d_out, d_in, 6, 302, device=dev)
+    pm = spax.alloc_packed(d_out, d_in, spax.FULL_BF16, device=dev)
+    spax.spax_pack_weights(W, spax.FULL_BF16, pm)
+    torch.cuda.synchronize()
+    del W
+    x = synth.laplace((d_in,), 6, 312, device=dev)
+    tier = torch.empty(d_in, dtype=torch.uint8, device=dev)
+    fi = torch.empty(d_in, dtype=torch.int32, device=dev)
+    ai = torch.empty(d_in, dtype=torch.int32, device=dev)
+    cnt = torch.empty(4, dtype=torch.int32, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    y = torch.empty(d_out, device=dev)
+    ws = spax.alloc_workspace(spax.OP_TIERED_GEMV, d_out, d_in, device=dev)
+    spax.spax_build_mask(x, spax.mask_params(spax.MASK_TOPK, k_full=0, k_approx=d_in), tier, fi, ai,
+                         cnt, st)
+    for _ in range(4):
+        spax.spax_tiered_gemv(pm, x, fi, ai, cnt, y, st, ws)
+    torch.cuda.synchronize()
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())}")
+    return 0
 
 
 def run_host_link(args, dev):
@@ -894,6 +1114,9 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=24)
     ap.add_argument("--ref-tokens", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-case", action="store_true",
+                    help="profiling aid: run only the list-driven all-2-bit GEMV on 22016x4096 (one "
+                         "mask launch, then 4 GEMV launches on one L2-resident copy); no JSON line")
     ap.add_argument("--host-link-only", action="store_true",
                     help="profiling aid: run only the host-link offload measurement (pools in "
                          "page-locked host memory) and print its JSON; not the benchmark line")
@@ -909,6 +1132,9 @@ def main():
     try:
         if args.impl == "reference":
             return run_reference(args, rank, world)
+        if args.decode_case:
+            torch.cuda.set_device(local)
+            return run_decode_case(args, torch.device("cuda", local)) if rank == 0 else 0
         if args.host_link_only:
             torch.cuda.set_device(local)
             if rank == 0:

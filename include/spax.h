@@ -353,6 +353,32 @@ spax_status spax_gemv_plan(int op, int d_out, int d_in, int full_fmt, int32_t* h
                            int32_t* h_row_tile);
 
 /*
+ * spax_output_change — d_acc[0] += Σ_i (y_i - y_ref_i)^2 and d_acc[1] += Σ_i y_ref_i^2 over the n
+ * entries of two device vectors, in fp64, by one CTA in a fixed order (the same bits on every
+ * run). d_acc: two doubles on the device, accumulated into (the caller zeroes them).
+ * Source: TopK-Guided §2.2 (block sensitivity as the output change at a probe sparsity).
+ */
+spax_status spax_output_change(const float* d_y, const float* d_y_ref, int n, double* d_acc,
+                               void* stream);
+
+/*
+ * spax_probe_sensitivity — offline: how far one matrix's output moves when its input is
+ * sparsified to the probe sparsity s̄ = s_probe_bp / 1e4 (TopK-Guided §2.2: each block's
+ * sensitivity is measured as its output change at a probe sparsity; the budgets then follow from
+ * spax_block_budgets). For each calibration token x_t (row t of d_X, row-major [n_tok][d_in]):
+ * y_ref = the masked GEMV with every column in full (the matrix's own full-tier format) and y =
+ * the masked GEMV with the TopK rule k_full = d_in - floor(s̄ d_in + 1/2), k_approx = 0 (the
+ * smallest |x| skipped, the rest in full); then spax_output_change(y, y_ref) into d_acc. A
+ * block's sensitivity is sqrt(Σ_m acc0_m / Σ_m acc1_m) over its matrices m. At s̄ = 0 both
+ * products take the same columns in the same order, so acc0 gains exactly 0.
+ * d_y2: device scratch of 2 * d_out floats (the second half 16-byte aligned); d_ws / ws_bytes:
+ * the tiered GEMV's workspace (zeroed before first use). Launches 3 * n_tok kernels on stream.
+ */
+spax_status spax_probe_sensitivity(const spax_packed* h_W, const float* d_X, int n_tok,
+                                   int s_probe_bp, float* d_y2, double* d_acc, int32_t* d_status,
+                                   void* d_ws, size_t ws_bytes, void* stream);
+
+/*
  * spax_block_budgets — host-only: sensitivity-aware per-block sparsity (TopK-Guided §2.2:
  * above-average-sensitivity blocks get less sparsity, λ sets the redistribution, results are
  * clamped to [lo, hi], the global budget is kept). With σ̄ the mean of h_sens:

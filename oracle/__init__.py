@@ -263,6 +263,34 @@ def dense_gemv(W_bits, x, rows=None):
     return y
 
 
+def probe_sensitivity(full, approx, fmt, d_out, d_in, X, s_probe_bp: int):
+    """Output change of one matrix at the probe sparsity s = s_probe_bp / 1e4 over calibration
+    tokens (TopK-Guided §2.2: block sensitivity measured at a probe sparsity). For each row x of X:
+    y_ref = the tiered product with every column full, y = the product with the TopK rule
+    k_full = d_in - floor(s d_in + 1/2), k_approx = 0. Returns (sum (y - y_ref)^2, sum y_ref^2)
+    in fp64, both summed over tokens and rows."""
+    X = np.atleast_2d(_c(X, np.float32))
+    skip = (int(s_probe_bp) * d_in + 5000) // 10000
+    all_full = np.full(d_in, 2, np.uint8)
+    a0 = a1 = 0.0
+    for x in X:
+        st, tier, _, _, _ = tiers(x, MODE_TOPK, k_full=d_in - skip, k_approx=0)
+        if st != OK:
+            raise ValueError("non-finite calibration token")
+        y = tiered_gemv(full, approx, fmt, d_out, d_in, x, tier)
+        y_ref = tiered_gemv(full, approx, fmt, d_out, d_in, x, all_full)
+        a0 += float(np.sum((y - y_ref) ** 2))
+        a1 += float(np.sum(y_ref ** 2))
+    return a0, a1
+
+
+def block_sensitivity(accs):
+    """A block's sensitivity from its matrices' (change, reference) sums: sqrt(sum a0 / sum a1)."""
+    a0 = sum(a[0] for a in accs)
+    a1 = sum(a[1] for a in accs)
+    return float(np.sqrt(a0 / a1)) if a1 > 0 else 0.0
+
+
 # ----------------------------------------------------------------------------- calibration etc.
 
 def calibrate(X, s_skip_bp: int, s_below_full_bp: int):
