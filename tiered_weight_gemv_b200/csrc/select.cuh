@@ -35,6 +35,8 @@
 // 2048-bin scan per boundary take the place of passes 1 to 2b whenever the guess holds.
 #pragma once
 
+#include <cstddef>
+
 #include "common.cuh"
 
 namespace spax {
@@ -52,7 +54,7 @@ struct Boundary {
   uint32_t lo, eqv, rem;
 };
 
-struct SelectSmem {
+struct alignas(16) SelectSmem {
   uint32_t hist[kSelBins];
   uint32_t ha[2][1024];  // bits 18..9 under each boundary's 12-bit prefix
   uint32_t hb[2][512];   // bits 8..0 under a 22-bit prefix (when pass 2 leaves V open)
@@ -85,11 +87,18 @@ __device__ __forceinline__ long long guided_clip(long long n, long long d, long 
 }
 
 // Zero what the selection accumulates into (all threads; may run before the wait on the
-// preceding kernel).
+// preceding kernel). hist, ha and hb are one run of words, cleared with 16-byte stores.
 __device__ __forceinline__ void select_zero(SelectSmem& S) {
-  for (int i = threadIdx.x; i < kSelBins; i += kSelThreads) S.hist[i] = 0u;
-  for (int i = threadIdx.x; i < 2 * 1024; i += kSelThreads) (&S.ha[0][0])[i] = 0u;
-  for (int i = threadIdx.x; i < 2 * 512; i += kSelThreads) (&S.hb[0][0])[i] = 0u;
+  constexpr int kZeroQuads = (kSelBins + 2 * 1024 + 2 * 512) / 4;
+  static_assert(offsetof(SelectSmem, ha) == kSelBins * 4 &&
+                    offsetof(SelectSmem, hb) == (kSelBins + 2 * 1024) * 4 && kSelBins % 4 == 0,
+                "hist, ha and hb must be one run of 16-byte quads");
+  uint4* z = reinterpret_cast<uint4*>(S.hist);
+#pragma unroll
+  for (int k = 0; k < (kZeroQuads + kSelThreads - 1) / kSelThreads; ++k) {
+    const int i = (int)threadIdx.x + k * kSelThreads;
+    if (i < kZeroQuads) z[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
   if (threadIdx.x < 4) S.stat[threadIdx.x] = 0u;
   if (threadIdx.x < 8) S.hint[threadIdx.x] = 0u;
 }
@@ -735,13 +744,15 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, SelectSmem& S, u
   }
   if (lane == 31) S.wscan[wid] = incl;
   __syncthreads();
-  uint32_t base = 0, all = 0;
+  // the warp totals, one per lane, by a second shuffle scan; this warp's base from lane wid - 1
+  uint32_t t = lane < kSelWarps ? S.wscan[lane] : 0u;
 #pragma unroll
-  for (int w = 0; w < kSelWarps; ++w) {
-    const uint32_t s = S.wscan[w];
-    base += w < wid ? s : 0u;
-    all += s;
+  for (int o = 1; o < kSelWarps; o <<= 1) {
+    const uint32_t n = __shfl_up_sync(0xffffffffu, t, o);
+    if (lane >= o) t += n;
   }
+  const uint32_t base = wid ? __shfl_sync(0xffffffffu, t, wid - 1) : 0u;
+  const uint32_t all = __shfl_sync(0xffffffffu, t, kSelWarps - 1);
   if (kReuse) __syncthreads();  // S.wscan may be reused right after
   *total = all;
   return base + incl - v;
