@@ -154,11 +154,12 @@ spax_status spax_build_mask(const float* x, int d_in, const spax_mask_params* p,
 size_t spax_workspace_bytes(int op, int d_out, int d_in) {
   if (op == SPAX_OP_CALIBRATE) return calibrate_ws_bytes();
   if (op != SPAX_OP_TIERED_GEMV && op != SPAX_OP_DENSE_GEMV) return 0;
-  // enough for either full-tier format (their row tiles, hence splits, differ)
+  // enough for either full-tier format
   GemvPlan pb, pi;
   const int sms = sm_count_current_device();
-  if (!make_gemv_plan(d_out, d_in, SPAX_FULL_BF16, sms, &pb)) return 0;
-  if (!make_gemv_plan(d_out, d_in, SPAX_FULL_INT4_G128, sms, &pi)) return 0;
+  const bool dense = op == SPAX_OP_DENSE_GEMV;
+  if (!make_gemv_plan(d_out, d_in, SPAX_FULL_BF16, sms, dense, &pb)) return 0;
+  if (!make_gemv_plan(d_out, d_in, SPAX_FULL_INT4_G128, sms, dense, &pi)) return 0;
   return pb.ws_bytes > pi.ws_bytes ? pb.ws_bytes : pi.ws_bytes;
 }
 
@@ -168,7 +169,7 @@ spax_status spax_gemv_plan(int op, int d_out, int d_in, int full_fmt, int32_t* s
   GemvPlan pl;
   const int sms = sm_count_current_device();
   if (sms < 1) return SPAX_ERR_CUDA;
-  if (!make_gemv_plan(d_out, d_in, full_fmt, sms, &pl)) return SPAX_ERR_SHAPE;
+  if (!make_gemv_plan(d_out, d_in, full_fmt, sms, op == SPAX_OP_DENSE_GEMV, &pl)) return SPAX_ERR_SHAPE;
   if (splits) *splits = pl.S;
   if (row_tile) *row_tile = pl.R;
   return SPAX_OK;
@@ -187,7 +188,7 @@ static spax_status gemv_common(const void* full, const void* approx, int full_fm
   const int sms = sm_count_current_device();
   if (sms < 1) return SPAX_ERR_CUDA;
   GemvPlan pl;
-  if (!make_gemv_plan(d_out, d_in, full_fmt, sms, &pl)) return SPAX_ERR_SHAPE;
+  if (!make_gemv_plan(d_out, d_in, full_fmt, sms, dense, &pl)) return SPAX_ERR_SHAPE;
   if (drop_splits && pl.S <= drop_splits) return SPAX_ERR_SHAPE;
   if (!ws || ws_bytes < pl.ws_bytes) return SPAX_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(ws) & 255u) return SPAX_ERR_ARG;
@@ -235,7 +236,7 @@ static spax_status masked_gemv_common(const spax_packed* W, const float* x, bool
   const int sms = sm_count_current_device();
   if (sms < 1) return SPAX_ERR_CUDA;
   GemvPlan pl;
-  if (!make_gemv_plan(W->d_out, W->d_in, W->full_fmt, sms, &pl)) return SPAX_ERR_SHAPE;
+  if (!make_gemv_plan(W->d_out, W->d_in, W->full_fmt, sms, false, &pl)) return SPAX_ERR_SHAPE;
   if (masked_gemv_smem_bytes(pl, W->d_in) > kMaskedGemvSmemLimit) return SPAX_ERR_SHAPE;
   if (!ws || ws_bytes < pl.ws_bytes) return SPAX_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(ws) & 255u) return SPAX_ERR_ARG;

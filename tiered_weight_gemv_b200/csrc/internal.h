@@ -18,7 +18,8 @@ struct GemvPlan {
 };
 
 int sm_count_current_device();  // cached per device; 0 on error
-bool make_gemv_plan(int d_out, int d_in, int full_fmt, int sm_count, GemvPlan* plan);
+// dense: the plan of the dense GEMV (its own row-tile rule); otherwise the tiered kernels'.
+bool make_gemv_plan(int d_out, int d_in, int full_fmt, int sm_count, bool dense, GemvPlan* plan);
 
 struct GemvLaunch {
   const void* full;
