@@ -379,6 +379,16 @@ spax_status spax_probe_sensitivity(const spax_packed* h_W, const float* d_X, int
                                    void* d_ws, size_t ws_bytes, void* stream);
 
 /*
+ * Host-only, no CUDA call: the plan of op for a GPU with sm_count SMs (the split count S, the row
+ * tile R and the workspace bytes), by the same rule the calls use on the current device. For
+ * sizing workspaces for another GPU model, and for checking a shape against
+ * spax_fixed_scratch_bytes(): spax_tiered_gemv_fixed_scratch rejects exactly the shapes whose
+ * SPAX_OP_TIERED_GEMV plan needs more workspace than that (SPAX_ERR_WORKSPACE).
+ */
+spax_status spax_gemv_plan_sms(int op, int d_out, int d_in, int full_fmt, int sm_count,
+                               int32_t* h_splits, int32_t* h_row_tile, size_t* h_ws_bytes);
+
+/*
  * spax_block_budgets — host-only: sensitivity-aware per-block sparsity (TopK-Guided §2.2:
  * above-average-sensitivity blocks get less sparsity, λ sets the redistribution, results are
  * clamped to [lo, hi], the global budget is kept). With σ̄ the mean of h_sens:

@@ -146,3 +146,33 @@ def test_device_calls_validate_arguments_before_any_launch():
                                        None) == spax.ERR_ARG  # a target above 100%
     assert L.spax_calibrate_thresholds(dummy, 4, 16, 3000, 6000, dummy, dummy, None, 1 << 20,
                                        None) == spax.ERR_WORKSPACE
+
+
+def test_plan_for_an_sm_count_and_the_fixed_scratch_bound():
+    """spax_gemv_plan_sms (no CUDA call) gives the plans the calls make. On 148 SMs no tiered plan
+    needs more than the fixed scratch array (4 MiB): a plan with splits stays within
+    148 x 2048 x 8 bytes. On a hypothetical 1184-SM part the same rule asks for more for some
+    shapes, which is exactly the condition under which spax_tiered_gemv_fixed_scratch returns
+    SPAX_ERR_WORKSPACE."""
+    fixed = spax.spax_fixed_scratch_bytes()
+    assert fixed == 4 << 20
+    worst = 0
+    for d_out in list(range(128, 40000, 128)) + [57344, 1 << 20]:
+        S, R, ws = spax.spax_gemv_plan_sms(spax.OP_TIERED_GEMV, d_out, 4096, spax.FULL_BF16, 148)
+        T = -(-d_out // R)
+        assert R in (512, 1024, 2048) and S >= 1
+        if S > 1:
+            assert T * S <= 148  # one wave
+            assert ws >= S * d_out * 8 and ws <= 148 * 2048 * 8 + 255
+        worst = max(worst, ws)
+    assert worst <= fixed
+    S, R, ws = spax.spax_gemv_plan_sms(spax.OP_TIERED_GEMV, 8192, 8192, spax.FULL_BF16, 1184)
+    assert S * (-(-8192 // R)) <= 1184 and ws > fixed  # the case the fixed-scratch call rejects
+    # the block's plans on B200 (the tiered rule and the dense rule differ)
+    assert spax.spax_gemv_plan_sms(spax.OP_TIERED_GEMV, 12288, 4096, 0, 148)[:2] == (6, 512)
+    assert spax.spax_gemv_plan_sms(spax.OP_TIERED_GEMV, 22016, 4096, 0, 148)[:2] == (3, 512)
+    assert spax.spax_gemv_plan_sms(spax.OP_DENSE_GEMV, 22016, 4096, 0, 148)[:2] == (13, 2048)
+    with pytest.raises(spax.SpaxError):
+        spax.spax_gemv_plan_sms(spax.OP_TIERED_GEMV, 100, 4096, 0, 148)  # d_out % 128 != 0
+    with pytest.raises(spax.SpaxError):
+        spax.spax_gemv_plan_sms(spax.OP_TIERED_GEMV, 4096, 4096, 0, 0)

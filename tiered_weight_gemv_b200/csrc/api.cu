@@ -175,6 +175,19 @@ spax_status spax_gemv_plan(int op, int d_out, int d_in, int full_fmt, int32_t* s
   return SPAX_OK;
 }
 
+spax_status spax_gemv_plan_sms(int op, int d_out, int d_in, int full_fmt, int sm_count,
+                               int32_t* splits, int32_t* row_tile, size_t* ws_bytes) {
+  if (op != SPAX_OP_TIERED_GEMV && op != SPAX_OP_DENSE_GEMV) return SPAX_ERR_ARG;
+  if (sm_count < 1) return SPAX_ERR_ARG;
+  GemvPlan pl;
+  if (!make_gemv_plan(d_out, d_in, full_fmt, sm_count, op == SPAX_OP_DENSE_GEMV, &pl))
+    return SPAX_ERR_SHAPE;
+  if (splits) *splits = pl.S;
+  if (row_tile) *row_tile = pl.R;
+  if (ws_bytes) *ws_bytes = pl.ws_bytes;
+  return SPAX_OK;
+}
+
 static spax_status gemv_common(const void* full, const void* approx, int full_fmt, const float* x,
                                const int32_t* fidx, const int32_t* aidx, const int32_t* counts,
                                float* y, int d_out, int d_in, int32_t* status, void* ws,

@@ -124,7 +124,7 @@ spax_status spax_tiered_gemv_fixed_scratch(const spax_packed* W, const float* x,
   if (sms < 1) return SPAX_ERR_CUDA;
   GemvPlan pl;
   if (!make_gemv_plan(W->d_out, W->d_in, W->full_fmt, sms, false, &pl)) return SPAX_ERR_SHAPE;
-  if (pl.ws_bytes > kFixedScratchBytes) return SPAX_ERR_WORKSPACE;
+  if (pl.ws_bytes > kFixedScratchBytes) return SPAX_ERR_WORKSPACE;  // see spax_gemv_plan_sms
   uint8_t* scratch = fixed_scratch_current_device();
   if (!scratch) return SPAX_ERR_CUDA;
   GemvLaunch a;

@@ -77,6 +77,7 @@ _SIGS = {
                                       ctypes.c_uint64, _P], _I),
     "spax_workspace_bytes": ([_I, _I, _I], _Z),
     "spax_gemv_plan": ([_I, _I, _I, _I, _P, _P], _I),
+    "spax_gemv_plan_sms": ([_I, _I, _I, _I, _I, _P, _P, _P], _I),
     "spax_block_budgets": ([_P, _I, ctypes.c_double, ctypes.c_double, ctypes.c_double,
                             ctypes.c_double, _P], _I),
     "spax_weight_bytes": ([_I, _I, ctypes.c_int64, ctypes.c_int64], ctypes.c_uint64),
@@ -147,6 +148,15 @@ def spax_gemv_plan(op: int, d_out: int, d_in: int, full_fmt: int = FULL_BF16):
     _check("spax_gemv_plan", _lib.spax_gemv_plan(op, d_out, d_in, full_fmt, ctypes.byref(s),
                                                  ctypes.byref(r)))
     return int(s.value), int(r.value)
+
+
+def spax_gemv_plan_sms(op: int, d_out: int, d_in: int, full_fmt: int, sm_count: int):
+    """Host-only: (splits, row_tile, workspace bytes) of op's plan on a GPU with sm_count SMs."""
+    sp, r, w = ctypes.c_int32(0), ctypes.c_int32(0), ctypes.c_size_t(0)
+    _check("spax_gemv_plan_sms", _lib.spax_gemv_plan_sms(op, d_out, d_in, full_fmt, sm_count,
+                                                         ctypes.byref(sp), ctypes.byref(r),
+                                                         ctypes.byref(w)))
+    return int(sp.value), int(r.value), int(w.value)
 
 
 def spax_block_budgets(sens, s: float, lam: float, lo: float = 0.05, hi: float = 0.95):
