@@ -1,10 +1,11 @@
 """GPU parity on the five workloads at their full sizes, through the C ABI (needs a B200).
 
 Every matrix has its workload's real shape. Tiers, lists and counts are checked bit-exact on every
-token that runs; y is checked against the fp64 oracle on a sample of rows (every 61st row, plus the
-last rows of the ragged tile), within rel L2 <= 2e-3 and max abs <= 1e-2 * max|y|. The Llama-2-7B
-block runs exactly as bench.py runs it: the same seeded weights and inputs, the same plans, the
-kernels chained in a CUDA graph with programmatic dependent launch.
+token that runs; y is checked against the fp64 oracle on every row, within rel L2 <= 2e-3 and max
+abs <= 1e-2 * max|y|. The Llama-2-7B block runs as bench.py times it: the same seeded weights and
+inputs, the same plans, the headline's masked GEMV with its calibrated guesses of the TopK boundary
+keys, and the two-call path beside it, each chained in a CUDA graph with programmatic dependent
+launch.
 """
 import math
 import os
@@ -30,11 +31,6 @@ def _built(oracle_lib):
     return oracle_lib
 
 
-def sample_rows(d_out):
-    rows = np.arange(0, d_out, 61)
-    return np.unique(np.concatenate([rows, np.arange(max(0, d_out - 5), d_out)]))
-
-
 def k_of(frac, d):
     return int(math.floor(frac * d + 0.5))
 
@@ -45,10 +41,9 @@ class Site:
     def __init__(self, W, fmt):
         self.gm = GpuMatrix(W, fmt)
         self.pools = oracle.pack(bf16_bits(W), fmt)
-        self.rows = sample_rows(self.gm.d_out)
 
     def check(self, x, params):
-        rel, g = check_token(self.gm, self.pools, x, params, rows=self.rows)
+        rel, g = check_token(self.gm, self.pools, x, params)  # every row
         return rel, g
 
 
@@ -69,66 +64,94 @@ def test_single_projection_4096():
 # ------------------------------------------------------------------------- Llama-2-7B block
 
 def test_llama2_block_as_benchmarked():
+    """The 64-token Llama-2-7B block of the benchmark line, both ways it is timed: the headline's
+    one-launch masked GEMV (TopK with the calibrated boundary-key guesses, lists written) and the
+    two-call path (mask kernel, then the list-driven GEMV). Every token: tiers, lists and counts
+    equal the oracle's, and the two paths' y are identical bit for bit. Tokens 0, 17 and 63: y on
+    every row against the fp64 oracle."""
     sys.path.insert(0, ROOT)
     import bench
 
     n_tok = bench.N_TOKENS
     mats = bench.make_weights("cuda")
     xs = bench.make_inputs(mats, n_tok, "cuda")
+    guess = bench.calibrated_guesses(mats, "cuda")
     sites = {}
+
+    def outputs(d_out, d_in):
+        return dict(tier=torch.empty(n_tok, d_in, dtype=torch.uint8, device="cuda"),
+                    fidx=torch.empty(n_tok, d_in, dtype=torch.int32, device="cuda"),
+                    aidx=torch.empty(n_tok, d_in, dtype=torch.int32, device="cuda"),
+                    counts=torch.empty(n_tok, 4, dtype=torch.int32, device="cuda"),
+                    y=torch.empty(n_tok, d_out, dtype=torch.float32, device="cuda"))
+
     for name, d_out, d_in, _ in bench.SITES:
         kf, ka = bench.k_counts(d_in)
-        gm = GpuMatrix(mats[name], spax.FULL_BF16)
-        sites[name] = dict(gm=gm, prm=spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka),
-                           tier=torch.empty(n_tok, d_in, dtype=torch.uint8, device="cuda"),
-                           fidx=torch.empty(n_tok, d_in, dtype=torch.int32, device="cuda"),
-                           aidx=torch.empty(n_tok, d_in, dtype=torch.int32, device="cuda"),
-                           counts=torch.empty(n_tok, 4, dtype=torch.int32, device="cuda"),
-                           y=torch.empty(n_tok, d_out, dtype=torch.float32, device="cuda"))
+        sites[name] = dict(gm=GpuMatrix(mats[name], spax.FULL_BF16),
+                           prm=spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka),
+                           prm_guess=spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka,
+                                                      t_skip=guess[name][0],
+                                                      t_full=guess[name][1]),
+                           two=outputs(d_out, d_in), one=outputs(d_out, d_in))
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
 
-    def step():
+    def step_two_call():
         for t in range(n_tok):
             for name, *_ in bench.SITES:
-                s = sites[name]
-                spax.spax_build_mask(xs[name][t], s["prm"], s["tier"][t], s["fidx"][t],
-                                     s["aidx"][t], s["counts"][t], status)
-                spax.spax_tiered_gemv(s["gm"].pm, xs[name][t], s["fidx"][t], s["aidx"][t],
-                                      s["counts"][t], s["y"][t], status, s["gm"].ws)
+                s, o = sites[name], sites[name]["two"]
+                spax.spax_build_mask(xs[name][t], s["prm"], o["tier"][t], o["fidx"][t],
+                                     o["aidx"][t], o["counts"][t], status)
+                spax.spax_tiered_gemv(s["gm"].pm, xs[name][t], o["fidx"][t], o["aidx"][t],
+                                      o["counts"][t], o["y"][t], status, s["gm"].ws)
+
+    def step_masked():  # the headline step of bench.py
+        for t in range(n_tok):
+            for name, *_ in bench.SITES:
+                s, o = sites[name], sites[name]["one"]
+                spax.spax_masked_gemv(s["gm"].pm, xs[name][t], s["prm_guess"], o["y"][t], status,
+                                      s["gm"].ws, tier=o["tier"][t], full_idx=o["fidx"][t],
+                                      approx_idx=o["aidx"][t], counts=o["counts"][t])
 
     stream = torch.cuda.Stream()
-    with torch.cuda.stream(stream):
-        step()  # eager warm-up, then the same launches from a graph
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        step()
+    graphs = []
+    for step in (step_two_call, step_masked):
+        with torch.cuda.stream(stream):
+            step()  # eager warm-up, then the same launches from a graph
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step()
+        graphs.append(g)
     for s in sites.values():
-        s["y"].fill_(float("nan"))
+        for o in (s["two"], s["one"]):
+            o["y"].fill_(float("nan"))
+            o["counts"].fill_(-1)
     with torch.cuda.stream(stream):
-        g.replay()
+        for g in graphs:
+            g.replay()
     torch.cuda.synchronize()
     assert status.item() == 0
     for name, d_out, d_in, _ in bench.SITES:
         s = sites[name]
         pools = oracle.pack(bf16_bits(mats[name]), spax.FULL_BF16)
         X = xs[name].cpu().numpy()
-        tiers = s["tier"].cpu().numpy()
-        counts = s["counts"].cpu().numpy()
-        fidx, aidx = s["fidx"].cpu().numpy(), s["aidx"].cpu().numpy()
-        y = s["y"].cpu().numpy()
+        two = {k: v.cpu().numpy() for k, v in s["two"].items()}
+        one = {k: v.cpu().numpy() for k, v in s["one"].items()}
+        assert np.array_equal(one["y"], two["y"]), f"{name}: masked y differs from the two-call y"
         op = oracle_params(s["prm"])
         mode = op.pop("mode")
-        rows = sample_rows(d_out)
         for t in range(n_tok):
             st, t_o, f_o, a_o, c_o = oracle.tiers(X[t], mode, **op)
-            assert st == 0 and np.array_equal(counts[t], c_o), (name, t)
-            assert np.array_equal(tiers[t], t_o), (name, t)
-            assert np.array_equal(fidx[t, : c_o[0]], f_o) and np.array_equal(aidx[t, : c_o[1]], a_o)
+            assert st == 0, (name, t)
+            for r in (two, one):
+                assert np.array_equal(r["counts"][t], c_o), (name, t)
+                assert np.array_equal(r["tier"][t], t_o), (name, t)
+                assert np.array_equal(r["fidx"][t, : c_o[0]], f_o), (name, t)
+                assert np.array_equal(r["aidx"][t, : c_o[1]], a_o), (name, t)
             if t in (0, 17, n_tok - 1):
-                y_ref = oracle.tiered_gemv(*pools, spax.FULL_BF16, d_out, d_in, X[t], t_o, rows=rows)
-                check_y(y[t][rows], y_ref, f"{name} token {t}")
-        assert np.all(np.isfinite(y))
+                y_ref = oracle.tiered_gemv(*pools, spax.FULL_BF16, d_out, d_in, X[t], t_o)
+                check_y(one["y"][t], y_ref, f"{name} token {t}")
+        assert np.all(np.isfinite(one["y"]))
 
 
 # ------------------------------------------------------------------------- Llama-3-8B stack
