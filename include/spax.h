@@ -26,6 +26,9 @@
  *     malformed index lists, a pipeline wait that ran out) are written to *d_status (an int32
  *     on the device, may be NULL) as a spax_status value; the caller reads it after a sync.
  *     A kernel never clears *d_status; the caller zeroes it.
+ *   - Every pointer is aligned for its element type (4 bytes for float and int32, 8 for
+ *     double). Entry points that need more (16-byte pools and outputs, 256-byte workspaces)
+ *     say so and return SPAX_ERR_ARG when it does not hold.
  *   - Tier codes: 0 = skip, 1 = approximate (2-bit), 2 = full (original format).
  *   - Compacted column lists are in ascending column order.
  *

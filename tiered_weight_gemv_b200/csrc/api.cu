@@ -291,6 +291,7 @@ spax_status spax_masked_gemv_wina(const spax_packed* W, const float* x, const fl
 spax_status spax_output_change(const float* y, const float* y_ref, int n, double* acc,
                                void* stream) {
   if (!y || !y_ref || !acc) return SPAX_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(acc) & 7u) return SPAX_ERR_ARG;
   if (n < 1) return SPAX_ERR_SHAPE;
   return launch_status(launch_output_change(y, y_ref, n, acc, static_cast<cudaStream_t>(stream)));
 }
@@ -299,6 +300,7 @@ spax_status spax_probe_sensitivity(const spax_packed* W, const float* X, int n_t
                                    float* y2, double* acc, int32_t* status, void* ws,
                                    size_t ws_bytes, void* stream) {
   if (!W || !X || !y2 || !acc) return SPAX_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(acc) & 7u) return SPAX_ERR_ARG;
   if (n_tok < 1) return SPAX_ERR_SHAPE;
   if (s_probe_bp < 0 || s_probe_bp > 10000) return SPAX_ERR_ARG;
   const int d = W->d_in, d_out = W->d_out;
