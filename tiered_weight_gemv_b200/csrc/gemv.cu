@@ -372,8 +372,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
 
   // Asynchronous form for the bf16 path: the records of a batch are copied to staging buffer
   // buf by cp.async (no registers held) while the warp streams bf16 columns and decodes the
-  // previous batch; stage_ready waits for them and prepares the batch's coefficients. Lane k also
-  // fetches x of the batch's column k at issue, a batch ahead of its use.
+  // previous batch; stage_ready waits for them and prepares the batch's coefficients. Lane k
+  // fetches x of the batch's column k at issue, a batch ahead of its use, except in the masked
+  // int4 kernel, which measured faster taking it at ready (its x mostly sits in shared memory).
+  constexpr bool kXAtIssue = !FUSED || FMT == SPAX_FULL_BF16;
   float xn = 0.f;  // x of column `lane` of the batch in flight (0 for an invalid column)
   auto stage_issue = [&](int k0, int nb, int buf) {
     __syncwarp();  // every lane is done with what this buffer held
@@ -386,7 +388,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
                    : "memory");
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
-    if (lane < nb) {
+    if (kXAtIssue && lane < nb) {
       const int i = cg + CG * (k0 + lane), col = colA(i);
       xn = col >= 0 ? xA(i, col) : 0.f;  // an invalid column contributes zero
     }
@@ -395,7 +397,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
     asm volatile("cp.async.wait_all;" ::: "memory");
     __syncwarp();
     if (lane < nb) {
-      const float xk = xn;
+      float xk = xn;
+      if constexpr (!kXAtIssue) {
+        const int i = cg + CG * (k0 + lane), col = colA(i);
+        xk = col >= 0 ? xA(i, col) : 0.f;
+      }
       const uint4 sm = lds128(stage_s + kStage2Bytes * buf + 144 * lane + 128);
       const uint32_t w[4] = {sm.x, sm.y, sm.z, sm.w};
       float c[4];
@@ -564,7 +570,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
                        : "memory");
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
-        if (lane < nb) {
+        if (kXAtIssue && lane < nb) {
           const int i = cg + CG * (k0 + lane), col = colF(i);
           xn = col >= 0 ? xF(i, col) : 0.f;  // an invalid column contributes zero
         }
@@ -573,7 +579,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
         asm volatile("cp.async.wait_all;" ::: "memory");
         __syncwarp();
         if (lane < nb) {
-          const float xk = xn;
+          float xk = xn;
+          if constexpr (!kXAtIssue) {
+            const int i = cg + CG * (k0 + lane), col = colF(i);
+            xk = col >= 0 ? xF(i, col) : 0.f;
+          }
           // this half's four group scales: bf16 scales [4*half4, 4*half4 + 4) of the record
           const uint2 sw = lds64(stage_s + kStage4Bytes * buf + 272 * lane + 256 + 8 * half4);
           const uint32_t w[4] = {sw.x << 16, sw.x & 0xFFFF0000u, sw.y << 16, sw.y & 0xFFFF0000u};
