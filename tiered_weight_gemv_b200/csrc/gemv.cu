@@ -86,7 +86,6 @@ struct GemvParams {
   int keys_bytes;  // fused: x kept alive after the lists for the product (0: x shares the reused
                    // area with the GEMV's staging, and the kernel stashes its split's x values)
   int RG;          // row tile R = 512 * RG (1, 2 or 4)
-  int swiglu;      // fused only: x holds [g; u] and x_j = swiglu_x(g_j, u_j)
   float* x_out;    // fused swiglu only: the token's x (lead CTA; may be null)
   const float* norms;  // fused only, may be null: rank by the WINA score |x_j| * norms[j]
   unsigned long long wait_ns;  // bound of the split-K wait
@@ -154,14 +153,22 @@ __host__ __device__ inline size_t fused_select_bytes(int d) {
   return (sizeof(SelectSmem) + 15) / 16 * 16 + select_keys_bytes(d);
 }
 
-// FUSED: the kernel first runs the tier rule on x itself (select.cuh: every CTA computes the
-// same lists, staged in its shared memory), then reads its split's positions from there.
+// FUSED, the mask of the launch: 0 for the list-driven and dense kernels, which take their lists
+// from the caller. Otherwise the kernel first runs the tier rule itself (select.cuh: every CTA
+// computes the same lists, staged in its shared memory), then reads its split's positions from
+// there. The rule runs on x (kFusedX), on x = silu(g) * u formed from [g; u] (kFusedSwiglu), or on
+// the WINA score |x| * norm (kFusedScored). Each source is its own instance: code in this kernel
+// costs time even where it never runs (measured on the Llama-2-7B block: the plain instance 1.0 us
+// per token-layer faster without the other two sources' code).
+constexpr int kFusedX = 1, kFusedSwiglu = 2, kFusedScored = 3;
+
 // RGT: the row-tile factor fixed at compile time (1, 2, 4), or 0 for the launch's p.RG. The tiered
 // kernels take 0 (one image for every shape of a layer); the dense baseline, a pure stream that
 // gains from the constant, keeps one image per tile height.
-template <int RGT, int FMT, bool DENSE, bool FUSED>
+template <int RGT, int FMT, bool DENSE, int FUSED>
 __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const GemvParams p) {
   constexpr int U = kGemvU;
+  constexpr bool kSwiglu = FUSED == kFusedSwiglu, kScored = FUSED == kFusedScored;
   const int RG = RGT > 0 ? RGT : p.RG, R = 512 * RG, CG = kGemvWarps / RG;
   const int kSlotFloats = RG * 576;  // combine slot of a column group: 36 floats per 32 rows
   static_assert(FMT == SPAX_FULL_BF16 || !DENSE, "the dense GEMV reads the bf16 pool");
@@ -173,7 +180,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
   float* red = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(list) + p.list_bytes +
                                         p.keys_bytes);
   // fused, keys kept alive: x of every column for the product (null otherwise)
-  const uint32_t* x_live = (FUSED && p.keys_bytes && !p.norms)
+  const uint32_t* x_live = (FUSED && !kScored && p.keys_bytes)
                                ? reinterpret_cast<const uint32_t*>(reinterpret_cast<uint8_t*>(list) +
                                                                    p.list_bytes)
                                : nullptr;
@@ -213,9 +220,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
     select_zero(sel);
     pdl_wait();
     pdl_launch_dependents();
-    if (p.swiglu)
+    if constexpr (kSwiglu)
       select_fetch_swiglu(p.x, p.d_in, keys, tile == 0 && split == 0 ? p.x_out : nullptr);
-    else if (p.norms)
+    else if constexpr (kScored)
       select_fetch_scored(p.x, p.norms, p.d_in, keys);
     else
       select_fetch(p.x, p.d_in, keys);
@@ -257,8 +264,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
         // x shares the reused area: stash x of this split's first kGemvMeta positions of each
         // list in the metadata arrays (idle in this kernel) for the product (not with the WINA
         // score: its keys are scores, so the product reads x itself)
-        const int nfl = p.norms ? 0 : min(kGemvMeta, Kf > split ? (Kf - split + S - 1) / S : 0);
-        const int nal = p.norms ? 0 : min(kGemvMeta, Ka > split ? (Ka - split + S - 1) / S : 0);
+        const int nfl = kScored ? 0 : min(kGemvMeta, Kf > split ? (Kf - split + S - 1) / S : 0);
+        const int nal = kScored ? 0 : min(kGemvMeta, Ka > split ? (Ka - split + S - 1) / S : 0);
         for (int i = tid; i < nfl; i += kGemvThreads)
           reinterpret_cast<float*>(meta_col_f)[i] = __uint_as_float(keys[list[split + S * i]]);
         for (int i = tid; i < nal; i += kGemvThreads)
@@ -314,14 +321,14 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
   // same function the selection used)
   auto xval = [&](int col) -> float {
     if constexpr (FUSED) {
-      if (p.swiglu) return swiglu_x(__ldg(p.x + col), __ldg(p.x + p.d_in + col));
+      if constexpr (kSwiglu) return swiglu_x(__ldg(p.x + col), __ldg(p.x + p.d_in + col));
     }
     return __ldg(p.x + col);
   };
 
   // x of local position i of this split's approximate / full list: the fused kernel's stash
   // (first kGemvMeta positions), else x of the column
-  const int xs_lim = (FUSED && !p.norms && !p.keys_bytes) ? kGemvMeta : 0;  // stash positions
+  const int xs_lim = (FUSED && !kScored && !p.keys_bytes) ? kGemvMeta : 0;  // stash positions
   auto xA = [&](int i, int col) -> float {
     if constexpr (FUSED) {
       if (x_live) return __uint_as_float(x_live[col]);
@@ -791,7 +798,7 @@ bool make_gemv_plan(int d_out, int d_in, int full_fmt, int sm_count, bool dense,
   return true;
 }
 
-template <int RGT, int FMT, bool DENSE, bool FUSED>
+template <int RGT, int FMT, bool DENSE, int FUSED>
 static cudaError_t launch_one(const GemvParams& gp, const GemvPlan& pl, size_t smem,
                               cudaStream_t stream) {
   auto kern = tiered_gemv_kernel<RGT, FMT, DENSE, FUSED>;
@@ -800,7 +807,7 @@ static cudaError_t launch_one(const GemvParams& gp, const GemvPlan& pl, size_t s
   return launch_pdl(kern, dim3(pl.T, pl.S), dim3(kGemvThreads), smem, stream, gp);
 }
 
-template <int FMT, bool DENSE, bool FUSED>
+template <int FMT, bool DENSE, int FUSED>
 static cudaError_t launch_r(const GemvParams& gp, const GemvPlan& pl, size_t smem,
                             cudaStream_t stream) {
   if constexpr (DENSE) {
@@ -869,9 +876,9 @@ cudaError_t launch_gemv(const GemvLaunch& a, const GemvPlan& pl, cudaStream_t st
   GemvPlan grid = pl;  // the launched grid: every split, or (a failure-detection test) fewer
   grid.S = pl.S - a.drop_splits;
   if (grid.S < 1) return cudaErrorInvalidValue;
-  if (a.dense) return launch_r<SPAX_FULL_BF16, true, false>(gp, grid, smem, stream);
-  if (a.full_fmt == SPAX_FULL_BF16) return launch_r<SPAX_FULL_BF16, false, false>(gp, grid, smem, stream);
-  return launch_r<SPAX_FULL_INT4_G128, false, false>(gp, grid, smem, stream);
+  if (a.dense) return launch_r<SPAX_FULL_BF16, true, 0>(gp, grid, smem, stream);
+  if (a.full_fmt == SPAX_FULL_BF16) return launch_r<SPAX_FULL_BF16, false, 0>(gp, grid, smem, stream);
+  return launch_r<SPAX_FULL_INT4_G128, false, 0>(gp, grid, smem, stream);
 }
 
 cudaError_t launch_masked_gemv(const GemvLaunch& a, const spax_mask_params& prm, bool swiglu,
@@ -880,7 +887,6 @@ cudaError_t launch_masked_gemv(const GemvLaunch& a, const spax_mask_params& prm,
                                cudaStream_t stream) {
   GemvParams gp = make_params(a, pl);
   gp.prm = prm;
-  gp.swiglu = swiglu ? 1 : 0;
   gp.x_out = swiglu ? x_out : nullptr;
   gp.norms = swiglu ? nullptr : norms;
   gp.tier_out = tier;
@@ -891,8 +897,15 @@ cudaError_t launch_masked_gemv(const GemvLaunch& a, const spax_mask_params& prm,
   size_t kb;
   const size_t smem = masked_gemv_layout(a.d_in, &kb);
   gp.keys_bytes = (int)kb;
-  if (a.full_fmt == SPAX_FULL_BF16) return launch_r<SPAX_FULL_BF16, false, true>(gp, pl, smem, stream);
-  return launch_r<SPAX_FULL_INT4_G128, false, true>(gp, pl, smem, stream);
+  const bool bf16 = a.full_fmt == SPAX_FULL_BF16;
+  if (swiglu)
+    return bf16 ? launch_r<SPAX_FULL_BF16, false, kFusedSwiglu>(gp, pl, smem, stream)
+                : launch_r<SPAX_FULL_INT4_G128, false, kFusedSwiglu>(gp, pl, smem, stream);
+  if (norms)
+    return bf16 ? launch_r<SPAX_FULL_BF16, false, kFusedScored>(gp, pl, smem, stream)
+                : launch_r<SPAX_FULL_INT4_G128, false, kFusedScored>(gp, pl, smem, stream);
+  return bf16 ? launch_r<SPAX_FULL_BF16, false, kFusedX>(gp, pl, smem, stream)
+              : launch_r<SPAX_FULL_INT4_G128, false, kFusedX>(gp, pl, smem, stream);
 }
 
 }  // namespace spax
