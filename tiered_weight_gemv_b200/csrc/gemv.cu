@@ -237,7 +237,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
     Boundary B[2];
     const bool bad = select_rule(p.prm, p.d_in, keys, sel, &n1, &n2, B);
     const bool lead = tile == 0 && split == 0;
-    if (bad) {  // non-finite x: every tier 0, empty lists, y = 0
+    if (__builtin_expect(bad, 0)) {  // non-finite x: every tier 0, empty lists, y = 0
       Kf = 0;
       Ka = 0;
       if (lead) {

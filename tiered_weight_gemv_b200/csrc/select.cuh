@@ -615,7 +615,8 @@ __device__ __forceinline__ int select_topk_guessed(const spax_mask_params& prm, 
   };
   // rank K lies in the window iff the scan from the top finds it before the window's bottom
   block_find_pair<kGuessBins>(h0, h1, act0, act1, K0, K1, A0, A1, 0u, 0u, 0, S);
-  if ((act0 && S.sel[0][0] == kNoKey) || (act1 && S.sel[1][0] == kNoKey)) return unwind();
+  if (__builtin_expect((act0 && S.sel[0][0] == kNoKey) || (act1 && S.sel[1][0] == kNoKey), 0))
+    return unwind();
   // ---- per boundary: the bin of rank K, the count above it and in it ----
   uint32_t base[2], above[2], cnt[2];
   bool need[2];
@@ -650,7 +651,7 @@ __device__ __forceinline__ int select_topk_guessed(const spax_mask_params& prm, 
     }
   }
   if (!need[0] && !need[1]) return 1;
-  if (crowded) return unwind();
+  if (__builtin_expect(crowded, 0)) return unwind();
   // ---- gather the keys of each unresolved bin, then rank them (one warp per boundary) ----
   const uint32_t g0 = base[0], g1 = base[1];
   const uint32_t gw0 = need[0] ? (1u << sh0) : 0u, gw1 = need[1] ? (1u << sh1) : 0u;
@@ -671,7 +672,8 @@ __device__ __forceinline__ int select_topk_guessed(const spax_mask_params& prm, 
   }
   __syncthreads();
   // the gathered counts equal the histogram's by construction; anything else is not trusted
-  if ((need[0] && S.hint[5] != cnt[0]) || (need[1] && S.hint[6] != cnt[1])) return unwind();
+  if (__builtin_expect((need[0] && S.hint[5] != cnt[0]) || (need[1] && S.hint[6] != cnt[1]), 0))
+    return unwind();
   const int wid = tid >> 5;
   if (wid < 2 && (wid ? need[1] : need[0])) {  // warp t ranks boundary t's keys: V, gt < rem <= gt + eq
     const uint32_t c = wid ? cnt[1] : cnt[0], ab = wid ? above[1] : above[0];
@@ -716,7 +718,7 @@ __device__ __forceinline__ bool select_rule(const spax_mask_params& prm, int d,
                                             uint32_t* n1, uint32_t* n2, Boundary* B) {
   if (prm.mode == SPAX_MASK_TOPK) {
     const int g = select_topk_guessed(prm, d, keys, S, B);
-    if (g != 0) {
+    if (__builtin_expect(g != 0, 1)) {
       *n1 = *n2 = 0u;
       return g == 2;
     }
@@ -847,7 +849,7 @@ __device__ __forceinline__ void select_compact(const uint32_t* __restrict__ keys
       }
     }
   }
-  if (ties || ragged) {  // the general form: bounds checks and ordered equal keys
+  if (__builtin_expect(ties || ragged, 0)) {  // the general form: bounds checks and ordered equal keys
     for (int q = ties ? qa : qm; q < qb; ++q) {
       const uint4 v = ld_key4(kq, q);
       const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
