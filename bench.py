@@ -842,9 +842,63 @@ def run_llama2_70b_mlp(args, dev):
     return out
 
 
+def run_scaled_guess(args, dev):
+    """The headline's masked GEMV chain on tokens whose scale varies: each token of every site is
+    multiplied by its own LogUniform[0.5, 2] factor. Three ways to pass the boundary-key guess:
+    the headline's absolute quantiles (calibrated on unit-scale tokens, so most windows miss),
+    TOPK_SCALED with the same quantiles divided by the calibration tokens' mean |x| (the window
+    follows each token's mean), and no guess. All three select the same columns."""
+    from tiered_weight_gemv_b200 import spax, synth
+
+    n_tok = 16
+    steps, warmup = max(5, min(args.steps, 20)), args.warmup
+    stream = torch.cuda.Stream(device=dev)
+    mats = make_weights(dev)
+    xs = make_inputs(mats, n_tok, dev, seed=2)
+    cal = make_inputs(mats, N_CAL, dev, seed=1)
+    guess = calibrated_guesses(mats, dev)
+    sites = []
+    for name, d_out, d_in, tid in SITES:
+        scale = synth.log_uniform((n_tok,), 2, 700 + (tid or 0), 0.5, 2.0, device=dev)
+        x = (xs[name].double() * scale.double()[:, None]).float().contiguous()
+        mean_cal = float(cal[name].abs().double().mean())
+        kf, ka = k_counts(d_in)
+        pm = spax.alloc_packed(d_out, d_in, spax.FULL_BF16, device=dev)
+        spax.spax_pack_weights(mats[name], spax.FULL_BF16, pm)
+        reps = [pm] + [spax.PackedMatrix(d_out, d_in, spax.FULL_BF16, pm.full.clone(), pm.approx.clone())
+                       for _ in range(3)]
+        prms = {"absolute": spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka,
+                                             t_skip=guess[name][0], t_full=guess[name][1]),
+                "scaled": spax.mask_params(spax.MASK_TOPK_SCALED, k_full=kf, k_approx=ka,
+                                           t_skip=guess[name][0] / mean_cal,
+                                           t_full=guess[name][1] / mean_cal),
+                "none": spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka)}
+        sites.append(dict(x=x, reps=reps, descs=[r.desc() for r in reps], prms=prms,
+                          y=torch.empty(n_tok, d_out, device=dev),
+                          ws=spax.alloc_workspace(spax.OP_TIERED_GEMV, d_out, d_in, device=dev)))
+    del mats, cal
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    out = {"tokens": n_tok, "token_scale": "LogUniform[0.5, 2] per token and site"}
+    for how in ("absolute", "scaled", "none"):
+        def step(how=how):
+            for t in range(n_tok):
+                for sd in sites:
+                    r = t % len(sd["reps"])
+                    spax.spax_masked_gemv(sd["reps"][r], sd["x"][t], sd["prms"][how], sd["y"][t], st,
+                                          sd["ws"], desc=sd["descs"][r])
+        ms = _timed_graph(step, stream, steps, warmup)
+        out[f"{how}_guess_us_per_token_layer"] = round(ms * 1000 / n_tok, 3)
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} in the scaled-guess runs")
+    del sites
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_extras(args, dev):
     """Measurements beside the headline, on one GPU, each a CUDA graph timed like the headline."""
     out = {"dequant_vs_load": run_dequant(args, dev)}
+    out["guess_under_token_scale"] = run_scaled_guess(args, dev)
     out["llama3_8b_stack"] = run_llama3_stack(args, dev)
     out["llama2_70b_mlp_int4"] = run_llama2_70b_mlp(args, dev)
     out["host_link_offload"] = run_host_link(args, dev)

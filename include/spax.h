@@ -74,7 +74,12 @@ typedef enum {
 
 typedef enum { SPAX_FULL_BF16 = 0, SPAX_FULL_INT4_G128 = 1 } spax_full_fmt;
 
-typedef enum { SPAX_MASK_THRESHOLD = 0, SPAX_MASK_TOPK = 1, SPAX_MASK_GUIDED = 2 } spax_mask_mode;
+typedef enum {
+  SPAX_MASK_THRESHOLD = 0,
+  SPAX_MASK_TOPK = 1,
+  SPAX_MASK_GUIDED = 2,
+  SPAX_MASK_TOPK_SCALED = 3
+} spax_mask_mode;
 
 typedef enum { SPAX_OP_TIERED_GEMV = 0, SPAX_OP_DENSE_GEMV = 1, SPAX_OP_CALIBRATE = 2 } spax_op;
 
@@ -95,7 +100,14 @@ typedef enum { SPAX_OP_TIERED_GEMV = 0, SPAX_OP_DENSE_GEMV = 1, SPAX_OP_CALIBRAT
  *     windowed pass instead of the full search. Any value is accepted (0, a negative, NaN or
  *     Inf means no guess), and the selected columns never depend on it. A guess that misses
  *     costs that pass (about 2 us per launch) on top of the full search, so pass none where
- *     the token-to-token scale of x varies by more than the window.
+ *     the token-to-token scale of x varies by more than the window (or use TOPK_SCALED).
+ *   TOPK_SCALED: TOPK (the same columns, lists and counts, counts[2] = counts[3] = 0) whose
+ *     guesses t_full and t_skip are multiples of the token's mean key: the mean of |x| over the
+ *     d_in columns (of the WINA score in spax_masked_gemv_wina). The kernels multiply them by
+ *     that mean (one block reduction, fp32, fixed order) before the windowed pass, so the
+ *     guess follows the token's scale. Calibrate the multiples as the quantiles divided by the
+ *     mean |x| of the calibration tokens. Same requirements as TOPK. Not a rule of the pages:
+ *     it only changes how fast the boundaries are found.
  *   GUIDED (TopK-Guided §2.1): the natural counts n1 = #{|x| < t_skip} and n2 = #{|x| < t_full}
  *     are clipped into the bands [ceil((s-δ)d), floor((s+δ)d)] around the skip target
  *     s = s_skip_bp/1e4 and the skip-or-approximate target s = s_below_full_bp/1e4

@@ -73,7 +73,8 @@ class GpuMatrix:
 
 def oracle_params(params) -> dict:
     mode = {spax.MASK_THRESHOLD: oracle.MODE_THRESHOLD, spax.MASK_TOPK: oracle.MODE_TOPK,
-            spax.MASK_GUIDED: oracle.MODE_GUIDED}[params.mode]
+            spax.MASK_GUIDED: oracle.MODE_GUIDED,
+            spax.MASK_TOPK_SCALED: oracle.MODE_TOPK}[params.mode]  # the same columns as TOPK
     return dict(mode=mode, t_skip=params.t_skip, t_full=params.t_full, k_full=params.k_full,
                 k_approx=params.k_approx, s_skip_bp=params.s_skip_bp,
                 s_below_full_bp=params.s_below_full_bp, delta_bp=params.delta_bp)

@@ -280,3 +280,123 @@ def test_guess_miss_stress(d):
         assert st.item() == 0
         _, t_o, _, _, _ = oracle.tiers(x, oracle.MODE_TOPK, k_full=kf, k_approx=ka)
         assert np.array_equal(tier.cpu().numpy(), t_o), f"masked GEMV token {tok}"
+
+
+def _masked(pm, d_out, d_in, x, prm, ws, norms=None, swiglu=False):
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = torch.full((d_out,), float("nan"), device="cuda")
+    tier = torch.full((d_in,), 7, dtype=torch.uint8, device="cuda")
+    fi = torch.full((d_in,), -1, dtype=torch.int32, device="cuda")
+    ai = torch.full((d_in,), -1, dtype=torch.int32, device="cuda")
+    c = torch.full((4,), -1, dtype=torch.int32, device="cuda")
+    kw = dict(tier=tier, full_idx=fi, approx_idx=ai, counts=c)
+    if swiglu:
+        spax.spax_masked_gemv_swiglu(pm, x, prm, y, st, ws, **kw)
+    elif norms is not None:
+        spax.spax_masked_gemv_wina(pm, x, norms, prm, y, st, ws, **kw)
+    else:
+        spax.spax_masked_gemv(pm, x, prm, y, st, ws, **kw)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    return [t.cpu().numpy() for t in (tier, fi, ai, c, y)]
+
+
+@pytest.mark.parametrize("d_out,d_in,fmt,src", [(4096, 4096, 0, "x"), (4096, 11008, 0, "x"),
+                                                (4096, 4096, 1, "x"), (4096, 4096, 0, "wina"),
+                                                (4096, 11008, 0, "swiglu"),
+                                                (8192, 20480, 0, "swiglu")])
+def test_scaled_guess_follows_token_scale(d_out, d_in, fmt, src):
+    """MASK_TOPK_SCALED: the guesses are multiples of the token's mean key, calibrated once on a
+    unit-scale token. Tokens scaled by 0.25 to 7.5 (SwiGLU: u scaled, so x = silu(g) * u scales
+    with it): on the host model of the window, the scaled
+    guess hits every token while the same guess taken as absolute keys misses the far scales; on
+    the GPU, the scaled rule gives the tiers, lists, counts and y of the unguessed TopK rule bit
+    for bit (and the oracle's tiers), through spax_build_mask and the masked GEMV. The sources:
+    plain x, the WINA score, and SwiGLU through the plain instance (4096 x 11008: x stays in shared
+    memory) and through its own instance (8192 x 20480)."""
+    W = synth.weight(d_out, d_in, 7, 9, device="cuda")
+    pm = spax.alloc_packed(d_out, d_in, fmt)
+    spax.spax_pack_weights(W, fmt, pm)
+    ws = spax.alloc_workspace(spax.OP_TIERED_GEMV, d_out, d_in)
+    norms = None
+    if src == "wina":
+        norms = torch.empty(d_in, device="cuda")
+        spax.spax_column_norms(W, norms)
+    del W
+    kf, ka = int(0.3 * d_in + 0.5), int(0.3 * d_in + 0.5)
+
+    def keys_of(v):  # the rule's keys on the host (fp32)
+        v = np.asarray(v, np.float32)
+        if src == "wina":
+            return np.abs(v) * norms.cpu().numpy()
+        if src == "swiglu":
+            return np.abs(oracle.swiglu(v[:d_in].astype(np.float64), v[d_in:].astype(np.float64)).astype(np.float32))
+        return np.abs(v)
+
+    n_in = 2 * d_in if src == "swiglu" else d_in
+    x0 = synth.laplace((n_in,), 70, 3).numpy()
+    k0 = keys_of(x0)
+    mean0 = float(np.mean(k0, dtype=np.float64))
+    rel_f, rel_s = kth_key(k0, kf) / mean0, kth_key(k0, kf + ka) / mean0
+    m = Mask(d_in) if src == "x" else None
+    missed_abs = 0
+    for i, scale in enumerate([0.25, 0.5, 1.0, 2.0, 4.0, 7.5]):
+        x = synth.laplace((n_in,), 71 + i, 3).numpy()
+        if src == "swiglu":  # x = silu(g) * u scales with u alone
+            x[d_in:] *= np.float32(scale)
+        else:
+            x *= np.float32(scale)
+        k = keys_of(x)
+        mean = float(np.mean(k, dtype=np.float64))
+        assert guess_path(k, kf, rel_f * mean) != "miss" and guess_path(k, kf + ka, rel_s * mean) != "miss"
+        missed_abs += "miss" in (guess_path(k, kf, rel_f * mean0), guess_path(k, kf + ka, rel_s * mean0))
+        xd = torch.from_numpy(x).cuda()
+        plain = spax.mask_params(spax.MASK_TOPK, k_full=kf, k_approx=ka)
+        scaled = spax.mask_params(spax.MASK_TOPK_SCALED, k_full=kf, k_approx=ka, t_full=rel_f,
+                                  t_skip=rel_s)
+        a = _masked(pm, d_out, d_in, xd, plain, ws, norms, src == "swiglu")
+        b = _masked(pm, d_out, d_in, xd, scaled, ws, norms, src == "swiglu")
+        for u, v in zip(a, b):
+            assert np.array_equal(u, v), f"scale {scale}: the scaled guess changed the result"
+        if src == "x":
+            _, t_o, _, _, c_o = oracle.tiers(x, oracle.MODE_TOPK, k_full=kf, k_approx=ka)
+            assert np.array_equal(b[0], t_o) and np.array_equal(b[3], c_o)
+            m.status.zero_()
+            spax.spax_build_mask(xd, scaled, m.tier, m.fidx, m.aidx, m.counts, m.status)
+            torch.cuda.synchronize()
+            assert m.status.item() == 0 and np.array_equal(m.tier.cpu().numpy(), t_o)
+            assert np.array_equal(m.counts.cpu().numpy(), c_o)
+    assert missed_abs >= 2  # the absolute guess misses the far scales
+
+
+def test_scaled_guess_edge_values():
+    """MASK_TOPK_SCALED with no usable guess (0, NaN, a negative multiple), an all-zero token and a
+    non-finite token: the results of the unguessed TopK rule, and SPAX_ERR_NONFINITE for the
+    last."""
+    d = 4096
+    m = Mask(d)
+    kf, ka = 1000, 1000
+    x = _laplace(d, 90)
+    _, t_o, f_o, a_o, c_o = oracle.tiers(x, oracle.MODE_TOPK, k_full=kf, k_approx=ka)
+    for tf, ts in [(0.0, 0.0), (float("nan"), 1.0), (-1.0, -2.0), (1e30, 1e-30)]:
+        prm = spax.mask_params(spax.MASK_TOPK_SCALED, k_full=kf, k_approx=ka, t_full=tf, t_skip=ts)
+        m.status.zero_()
+        spax.spax_build_mask(torch.from_numpy(x).cuda(), prm, m.tier, m.fidx, m.aidx, m.counts,
+                             m.status)
+        torch.cuda.synchronize()
+        assert m.status.item() == 0 and np.array_equal(m.tier.cpu().numpy(), t_o)
+        assert np.array_equal(m.counts.cpu().numpy(), c_o)
+    prm = spax.mask_params(spax.MASK_TOPK_SCALED, k_full=kf, k_approx=ka, t_full=1.2, t_skip=0.4)
+    z = np.zeros(d, np.float32)
+    _, t_z, _, _, c_z = oracle.tiers(z, oracle.MODE_TOPK, k_full=kf, k_approx=ka)
+    m.status.zero_()
+    spax.spax_build_mask(torch.from_numpy(z).cuda(), prm, m.tier, m.fidx, m.aidx, m.counts, m.status)
+    torch.cuda.synchronize()
+    assert m.status.item() == 0 and np.array_equal(m.tier.cpu().numpy(), t_z)
+    assert np.array_equal(m.counts.cpu().numpy(), c_z)
+    xn = x.copy()
+    xn[17] = np.inf
+    m.status.zero_()
+    spax.spax_build_mask(torch.from_numpy(xn).cuda(), prm, m.tier, m.fidx, m.aidx, m.counts, m.status)
+    torch.cuda.synchronize()
+    assert m.status.item() == spax.ERR_NONFINITE

@@ -123,7 +123,7 @@ spax_status spax_calibrate_thresholds(const float* calib_x, int n_tok, int d_in,
 
 // The rule's parameters for d_in columns (shared by the mask and the masked GEMV).
 static spax_status check_mask_params(const spax_mask_params& q, int d_in) {
-  if (q.mode == SPAX_MASK_TOPK) {
+  if (q.mode == SPAX_MASK_TOPK || q.mode == SPAX_MASK_TOPK_SCALED) {
     if (q.k_full < 0 || q.k_approx < 0 || (long long)q.k_full + q.k_approx > d_in)
       return SPAX_ERR_ARG;
   } else if (q.mode == SPAX_MASK_THRESHOLD || q.mode == SPAX_MASK_GUIDED) {

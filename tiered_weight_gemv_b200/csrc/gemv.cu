@@ -166,6 +166,9 @@ __host__ __device__ inline size_t fused_select_bytes(int d) {
 // layer's launches share one image that stays warm in the instruction caches (measured: the layer
 // with down fed from gate/up 68.8 -> 65.2 us); the SwiGLU instance serves the rest.
 constexpr int kFusedX = 1, kFusedSwiglu = 2, kFusedScored = 3;
+// Added to a source: the rule is TOPK_SCALED (the guesses of the boundary keys scale with the
+// token's mean key), its own instances so that the others carry none of its code.
+constexpr int kFusedScaled = 4;
 
 // RGT: the row-tile factor fixed at compile time (1, 2, 4), or 0 for the launch's p.RG. The tiered
 // kernels take 0 (one image for every shape of a layer); the dense baseline, a pure stream that
@@ -173,7 +176,8 @@ constexpr int kFusedX = 1, kFusedSwiglu = 2, kFusedScored = 3;
 template <int RGT, int FMT, bool DENSE, int FUSED>
 __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const GemvParams p) {
   constexpr int U = kGemvU;
-  constexpr bool kSwiglu = FUSED == kFusedSwiglu, kScored = FUSED == kFusedScored;
+  constexpr bool kSwiglu = (FUSED & 3) == kFusedSwiglu, kScored = (FUSED & 3) == kFusedScored;
+  constexpr bool kScaled = (FUSED & kFusedScaled) != 0;
   const int RG = RGT > 0 ? RGT : p.RG, R = 512 * RG, CG = kGemvWarps / RG;
   const int kSlotFloats = RG * 576;  // combine slot of a column group: 36 floats per 32 rows
   static_assert(FMT == SPAX_FULL_BF16 || !DENSE, "the dense GEMV reads the bf16 pool");
@@ -235,7 +239,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
       select_fetch(p.x, p.d_in, keys);
     uint32_t n1, n2;
     Boundary B[2];
-    const bool bad = select_rule(p.prm, p.d_in, keys, sel, &n1, &n2, B);
+    bool bad;
+    if constexpr (kScaled)
+      bad = select_rule(select_scaled_topk(p.prm, p.d_in, keys, sel), p.d_in, keys, sel, &n1, &n2, B);
+    else
+      bad = select_rule(p.prm, p.d_in, keys, sel, &n1, &n2, B);
     const bool lead = tile == 0 && split == 0;
     if (__builtin_expect(bad, 0)) {  // non-finite x: every tier 0, empty lists, y = 0
       Kf = 0;
@@ -888,6 +896,22 @@ cudaError_t launch_gemv(const GemvLaunch& a, const GemvPlan& pl, cudaStream_t st
   return launch_r<SPAX_FULL_INT4_G128, false, 0>(gp, grid, smem, stream);
 }
 
+// The masked instance of a FUSED value (source | kFusedScaled).
+template <int FMT>
+static cudaError_t launch_src(const GemvParams& gp, const GemvPlan& pl, size_t smem, int src,
+                              cudaStream_t stream) {
+  switch (src) {
+    case kFusedSwiglu: return launch_r<FMT, false, kFusedSwiglu>(gp, pl, smem, stream);
+    case kFusedScored: return launch_r<FMT, false, kFusedScored>(gp, pl, smem, stream);
+    case kFusedX | kFusedScaled: return launch_r<FMT, false, kFusedX | kFusedScaled>(gp, pl, smem, stream);
+    case kFusedSwiglu | kFusedScaled:
+      return launch_r<FMT, false, kFusedSwiglu | kFusedScaled>(gp, pl, smem, stream);
+    case kFusedScored | kFusedScaled:
+      return launch_r<FMT, false, kFusedScored | kFusedScaled>(gp, pl, smem, stream);
+    default: return launch_r<FMT, false, kFusedX>(gp, pl, smem, stream);
+  }
+}
+
 cudaError_t launch_masked_gemv(const GemvLaunch& a, const spax_mask_params& prm, bool swiglu,
                                float* x_out, const float* norms, uint8_t* tier, int32_t* full_idx,
                                int32_t* approx_idx, int32_t* counts, const GemvPlan& pl,
@@ -904,24 +928,20 @@ cudaError_t launch_masked_gemv(const GemvLaunch& a, const spax_mask_params& prm,
   size_t kb;
   const size_t smem = masked_gemv_layout(a.d_in, &kb);
   gp.keys_bytes = (int)kb;
-  const bool bf16 = a.full_fmt == SPAX_FULL_BF16;
   // A SwiGLU call whose product finds every x in shared memory (x kept alive, or each split's
   // positions within the stash for any count) runs the plain instance, which forms x in its
   // fetch: the layer's launches then share one image (warm in the instruction caches).
   const int per_split = (a.d_in + pl.S - 1) / pl.S;
-  if (swiglu && (kb != 0 || per_split <= kGemvMeta)) {
+  int src = kFusedX;
+  if (swiglu && (kb != 0 || per_split <= kGemvMeta))
     gp.fetch_swiglu = 1;
-    return bf16 ? launch_r<SPAX_FULL_BF16, false, kFusedX>(gp, pl, smem, stream)
-                : launch_r<SPAX_FULL_INT4_G128, false, kFusedX>(gp, pl, smem, stream);
-  }
-  if (swiglu)
-    return bf16 ? launch_r<SPAX_FULL_BF16, false, kFusedSwiglu>(gp, pl, smem, stream)
-                : launch_r<SPAX_FULL_INT4_G128, false, kFusedSwiglu>(gp, pl, smem, stream);
-  if (norms)
-    return bf16 ? launch_r<SPAX_FULL_BF16, false, kFusedScored>(gp, pl, smem, stream)
-                : launch_r<SPAX_FULL_INT4_G128, false, kFusedScored>(gp, pl, smem, stream);
-  return bf16 ? launch_r<SPAX_FULL_BF16, false, kFusedX>(gp, pl, smem, stream)
-              : launch_r<SPAX_FULL_INT4_G128, false, kFusedX>(gp, pl, smem, stream);
+  else if (swiglu)
+    src = kFusedSwiglu;
+  else if (norms)
+    src = kFusedScored;
+  if (prm.mode == SPAX_MASK_TOPK_SCALED) src |= kFusedScaled;
+  if (a.full_fmt == SPAX_FULL_BF16) return launch_src<SPAX_FULL_BF16>(gp, pl, smem, src, stream);
+  return launch_src<SPAX_FULL_INT4_G128>(gp, pl, smem, src, stream);
 }
 
 }  // namespace spax

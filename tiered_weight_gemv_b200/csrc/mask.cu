@@ -23,7 +23,10 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   select_fetch(x, d, keys);  // its barrier also orders the zeroing above
   uint32_t n1, n2;
   Boundary B[2];
-  if (select_rule(prm, d, keys, S, &n1, &n2, B)) {
+  const bool bad = prm.mode == SPAX_MASK_TOPK_SCALED
+                       ? select_rule(select_scaled_topk(prm, d, keys, S), d, keys, S, &n1, &n2, B)
+                       : select_rule(prm, d, keys, S, &n1, &n2, B);
+  if (bad) {
     for (int j = threadIdx.x; j < d; j += kSelThreads) tier[j] = 0;
     if (threadIdx.x == 0) {
       counts[0] = counts[1] = counts[2] = counts[3] = 0;
@@ -38,8 +41,9 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   if (threadIdx.x == 0) {
     counts[0] = (int32_t)nf;
     counts[1] = (int32_t)na;
-    counts[2] = prm.mode == SPAX_MASK_TOPK ? 0 : (int32_t)n1;
-    counts[3] = prm.mode == SPAX_MASK_TOPK ? 0 : (int32_t)n2;
+    const bool topk = prm.mode == SPAX_MASK_TOPK || prm.mode == SPAX_MASK_TOPK_SCALED;
+    counts[2] = topk ? 0 : (int32_t)n1;
+    counts[3] = topk ? 0 : (int32_t)n2;
   }
 }
 

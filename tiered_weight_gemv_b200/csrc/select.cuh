@@ -710,6 +710,36 @@ __device__ __forceinline__ int select_topk_guessed(const spax_mask_params& prm, 
   return 1;
 }
 
+// TOPK_SCALED -> TOPK: the guesses t_full and t_skip, given as multiples of the token's mean key
+// (mean |key| over the d columns), become keys (after a select_fetch*; all threads; one barrier).
+// A non-finite or zero mean leaves no usable guess, and the TopK search then runs unhinted (which
+// reports a non-finite key as the plain rule does).
+__device__ __forceinline__ spax_mask_params select_scaled_topk(const spax_mask_params& prm, int d,
+                                                              const uint32_t* __restrict__ keys,
+                                                              SelectSmem& S) {
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int nq = (d + 3) >> 2;
+  const uint4* kq = reinterpret_cast<const uint4*>(keys);
+  float sum = 0.f;  // the zero keys padding the last quad add nothing
+  for (int q = tid; q < nq; q += kSelThreads) {
+    const uint4 v = ld_key4(kq, q);
+    sum += (__uint_as_float(v.x) + __uint_as_float(v.y)) + (__uint_as_float(v.z) + __uint_as_float(v.w));
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) S.wsum[wid] = __float_as_uint(sum);  // free until the rule's first scan
+  __syncthreads();
+  float total = 0.f;
+#pragma unroll
+  for (int w = 0; w < kSelWarps; ++w) total += __uint_as_float(S.wsum[w]);
+  const float mean = total / (float)d;
+  spax_mask_params q = prm;
+  q.mode = SPAX_MASK_TOPK;
+  q.t_full = prm.t_full * mean;
+  q.t_skip = prm.t_skip * mean;
+  return q;
+}
+
 // The rule's two boundaries (after a select_fetch*; all threads; barriers inside): the guessed
 // TopK search when it applies and resolves, else pass 1 and select_boundaries. Returns true on a
 // non-finite key (B unset). n1, n2: the threshold counts (0 in TopK mode).

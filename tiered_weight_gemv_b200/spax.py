@@ -24,7 +24,7 @@ _lib = ctypes.CDLL(_LIB_PATH)
 OK = 0
 ERR_ARG, ERR_SHAPE, ERR_WORKSPACE, ERR_CUDA, ERR_NONFINITE, ERR_TIMEOUT, ERR_INDEX = 1, 2, 3, 4, 5, 6, 7
 FULL_BF16, FULL_INT4_G128 = 0, 1
-MASK_THRESHOLD, MASK_TOPK, MASK_GUIDED = 0, 1, 2
+MASK_THRESHOLD, MASK_TOPK, MASK_GUIDED, MASK_TOPK_SCALED = 0, 1, 2, 3
 OP_TIERED_GEMV, OP_DENSE_GEMV, OP_CALIBRATE = 0, 1, 2
 MASK_MAX_DIN = 32768
 
@@ -251,7 +251,8 @@ def mask_params(mode: int, *, t_skip=0.0, t_full=0.0, k_full=0, k_approx=0, s_sk
                 s_below_full_bp=0, delta_bp=0) -> spax_mask_params:
     """The rule's parameters (spax.h, spax_mask_params). In MASK_TOPK mode t_full / t_skip may
     carry a guess of the |x| at rank k_full / k_full + k_approx (calibrated quantiles); it only
-    speeds the selection up when it holds, and 0 means no guess."""
+    speeds the selection up when it holds, and 0 means no guess. MASK_TOPK_SCALED is the same
+    rule with the guesses given as multiples of the token's mean |x|."""
     return spax_mask_params(mode, t_skip, t_full, k_full, k_approx, s_skip_bp, s_below_full_bp,
                             delta_bp)
 
