@@ -229,19 +229,25 @@ __global__ void __launch_bounds__(kGemvThreads, 1) tiered_gemv_kernel(const Gemv
     select_zero(sel);
     pdl_wait();
     pdl_launch_dependents();
+    float x_mean = -1.f;  // TOPK_SCALED on plain x: the mean |x| gathered by the fetch
+    (void)x_mean;
     if constexpr (kSwiglu)
       select_fetch_swiglu(p.x, p.d_in, keys, tile == 0 && split == 0 ? p.x_out : nullptr);
     else if constexpr (kScored)
       select_fetch_scored(p.x, p.norms, p.d_in, keys);
     else if (p.fetch_swiglu)
       select_fetch_swiglu(p.x, p.d_in, keys, tile == 0 && split == 0 ? p.x_out : nullptr);
+    else if constexpr (kScaled)
+      x_mean = select_fetch_mean(p.x, p.d_in, keys, sel);  // the mean comes with the fetch
     else
       select_fetch(p.x, p.d_in, keys);
     uint32_t n1, n2;
     Boundary B[2];
     bool bad;
     if constexpr (kScaled)
-      bad = select_rule(select_scaled_topk(p.prm, p.d_in, keys, sel), p.d_in, keys, sel, &n1, &n2, B);
+      bad = select_rule(x_mean >= 0.f ? scaled_topk_params(p.prm, x_mean)
+                                      : select_scaled_topk(p.prm, p.d_in, keys, sel),
+                        p.d_in, keys, sel, &n1, &n2, B);
     else
       bad = select_rule(p.prm, p.d_in, keys, sel, &n1, &n2, B);
     const bool lead = tile == 0 && split == 0;

@@ -710,6 +710,53 @@ __device__ __forceinline__ int select_topk_guessed(const spax_mask_params& prm, 
   return 1;
 }
 
+// x[0, d) -> keys[] as select_fetch does, through registers, summing |x| on the way: returns the
+// mean |x| over the d columns (fp32, a fixed order). Ends with a barrier; S.wsum holds the warp
+// sums until the rule's first scan.
+__device__ __forceinline__ float select_fetch_mean(const float* __restrict__ x, int d,
+                                                   uint32_t* __restrict__ keys, SelectSmem& S) {
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int nfull = d >> 2;
+  float sum = 0.f;
+  if ((reinterpret_cast<uintptr_t>(x) & 15u) == 0) {
+    for (int q = tid; q < nfull; q += kSelThreads) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(x) + q);
+      reinterpret_cast<float4*>(keys)[q] = v;
+      sum += (fabsf(v.x) + fabsf(v.y)) + (fabsf(v.z) + fabsf(v.w));
+    }
+  } else {
+    for (int j = tid; j < 4 * nfull; j += kSelThreads) {
+      const float v = __ldg(x + j);
+      keys[j] = __float_as_uint(v);
+      sum += fabsf(v);
+    }
+  }
+  if (tid < 4 && (d & 3)) {
+    const int j = 4 * nfull + tid;
+    const float v = j < d ? __ldg(x + j) : 0.f;
+    keys[j] = __float_as_uint(v);
+    sum += fabsf(v);
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) S.wsum[wid] = __float_as_uint(sum);
+  __syncthreads();
+  float total = 0.f;
+#pragma unroll
+  for (int w = 0; w < kSelWarps; ++w) total += __uint_as_float(S.wsum[w]);
+  return total / (float)d;
+}
+
+// The TOPK_SCALED parameters as TOPK ones, given the token's mean key.
+__device__ __forceinline__ spax_mask_params scaled_topk_params(const spax_mask_params& prm,
+                                                               float mean) {
+  spax_mask_params q = prm;
+  q.mode = SPAX_MASK_TOPK;
+  q.t_full = prm.t_full * mean;
+  q.t_skip = prm.t_skip * mean;
+  return q;
+}
+
 // TOPK_SCALED -> TOPK: the guesses t_full and t_skip, given as multiples of the token's mean key
 // (mean |key| over the d columns), become keys (after a select_fetch*; all threads; one barrier).
 // A non-finite or zero mean leaves no usable guess, and the TopK search then runs unhinted (which
