@@ -132,6 +132,14 @@ def test_device_calls_validate_arguments_before_any_launch():
                              None) == spax.ERR_SHAPE
     bad_t = spax.mask_params(spax.MASK_THRESHOLD, t_skip=1.0, t_full=0.5)
     assert L.spax_build_mask(dummy, 16, bad_t, dummy, dummy, dummy, dummy, dummy, None) == spax.ERR_ARG
+    bad_scaled = spax.mask_params(spax.MASK_TOPK_SCALED, k_full=10, k_approx=10, t_full=1.2)
+    assert L.spax_build_mask(dummy, 16, bad_scaled, dummy, dummy, dummy, dummy, dummy,
+                             None) == spax.ERR_ARG
+    unknown = spax.mask_params(4, k_full=1, k_approx=1)  # no such rule
+    assert L.spax_build_mask(dummy, 16, unknown, dummy, dummy, dummy, dummy, dummy, None) == spax.ERR_ARG
+    # the fp64 accumulator of the sensitivity calls must be 8-byte aligned
+    assert L.spax_output_change(dummy, dummy, 16, dummy + 4, None) == spax.ERR_ARG
+    assert L.spax_output_change(dummy, dummy, 0, dummy, None) == spax.ERR_SHAPE
     assert L.spax_tiered_gemv(None, dummy, dummy, dummy, dummy, dummy, dummy, dummy, 1 << 20,
                               None) == spax.ERR_ARG
     desc = spax.spax_packed(100, 16, spax.FULL_BF16, 0, dummy, dummy)  # d_out % 128 != 0
