@@ -23,10 +23,11 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   select_fetch(x, d, keys);  // its barrier also orders the zeroing above
   uint32_t n1, n2;
   Boundary B[2];
-  const bool bad = prm.mode == SPAX_MASK_TOPK_SCALED
-                       ? select_rule(select_scaled_topk(prm, d, keys, S), d, keys, S, &n1, &n2, B)
-                       : select_rule(prm, d, keys, S, &n1, &n2, B);
-  if (bad) {
+  // TOPK_SCALED: its guesses become keys first (the token's mean key times the multiples), so
+  // the kernel holds one copy of the rule
+  const spax_mask_params rule =
+      prm.mode == SPAX_MASK_TOPK_SCALED ? select_scaled_topk(prm, d, keys, S) : prm;
+  if (select_rule(rule, d, keys, S, &n1, &n2, B)) {
     for (int j = threadIdx.x; j < d; j += kSelThreads) tier[j] = 0;
     if (threadIdx.x == 0) {
       counts[0] = counts[1] = counts[2] = counts[3] = 0;
